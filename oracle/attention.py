@@ -1,0 +1,104 @@
+"""Oracle: heterogeneous causal sliding-window attention.  TEST INFRASTRUCTURE ONLY.
+
+What the method computes
+------------------------
+"Mixture of Attention" project page, "Key findings" and the N x N causal
+attention figure of "Finding two": each head keeps a diagonal band of the
+causal attention matrix whose width is the head's own span S_h; everything
+outside the band is masked.  The blog walkthrough ("MoA: Mixture of Sparse
+Attention ...", section 2.1) builds the rule on a sliding-window mask, and
+its section 5 says the CUDA kernel applies the mask and aggregates attention.
+
+Written out, for batch b, query head h, query row i (0-based):
+
+    window(i)  = { j : i - S_h < j <= i, j >= 0 }        (S_h keys incl. i)
+    s_j        = scale * sum_k q[b,h,i,k] * k[b,g,j,k]      for j in window(i)
+    p_j        = exp(s_j - max_j s_j)
+    o[b,h,i,:] = sum_j p_j v[b,g,j,:] / sum_j p_j
+
+where g = h // (Hq // Hkv) is the key/value head that query head h reads
+(grouped-query attention; with Hq == Hkv, g == h).  Subtracting the row
+maximum leaves the result unchanged mathematically and keeps exp finite.
+
+Readings (listed in the design doc): the window holds S_h keys including the
+query's own position (S_h = 1 attends to itself only); no sink or global
+tokens; spans are per query head.
+
+Everything runs in numpy float64 on whatever values the caller passes
+(callers upcast the exact bf16 or fp32 values the GPU sees).
+"""
+
+import numpy as np
+
+
+def window(i, S):
+    """Inclusive key range [lo, hi] of query row ``i`` under span ``S``."""
+    if S < 1:
+        raise ValueError("span must be >= 1")
+    return max(0, i - S + 1), i
+
+
+def row_weights(q_i, K, lo, hi, scale):
+    """Softmax weights of one query row over keys lo..hi (float64 vector)."""
+    s = (np.asarray(K[lo:hi + 1], dtype=np.float64) @ np.asarray(q_i, dtype=np.float64)) * scale
+    p = np.exp(s - s.max())
+    return p / p.sum()
+
+
+def attend_row(q_i, K, V, lo, hi, scale):
+    """One output row: softmax over keys lo..hi applied to V[lo..hi]."""
+    w = row_weights(q_i, K, lo, hi, scale)
+    return w @ np.asarray(V[lo:hi + 1], dtype=np.float64)
+
+
+def prefill(q, k, v, spans, scale, rows=None):
+    """Windowed causal attention over a whole prompt.
+
+    q: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; spans: per query head (len Hq).
+    Returns float64 [B, Hq, N, d].  With ``rows`` given (an iterable of
+    (b, h, i) triples) returns a float64 array [len(rows), d] holding only
+    those output rows, for sampled checks at sizes where the full output
+    would take too long.
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if len(spans) != Hq:
+        raise ValueError("one span per query head")
+    G = Hq // Hkv
+    if rows is not None:
+        out = np.empty((len(rows), d), dtype=np.float64)
+        for n, (b, h, i) in enumerate(rows):
+            lo, hi = window(i, int(spans[h]))
+            out[n] = attend_row(q[b, h, i], k[b, h // G], v[b, h // G], lo, hi, scale)
+        return out
+    out = np.empty((B, Hq, N, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            K = np.asarray(k[b, g], dtype=np.float64)
+            V = np.asarray(v[b, g], dtype=np.float64)
+            S = int(spans[h])
+            for i in range(N):
+                lo, hi = window(i, S)
+                out[b, h, i] = attend_row(q[b, h, i], K, V, lo, hi, scale)
+    return out
+
+
+def in_window_flops(spans, N, d, B=1):
+    """Algorithmic FLOPs of prefill counting only in-window work.
+
+    Row i of head h touches min(i+1, S_h) keys; QK^T and PV each cost 2*d
+    flops per (row, key) pair, so the total is 4*d*sum_h sum_i min(i+1, S_h)
+    = 4*d*sum_h (S_h*N - S_h*(S_h-1)/2) for S_h <= N.
+    """
+    total = 0
+    for S in spans:
+        S = min(int(S), int(N))
+        pairs = S * N - S * (S - 1) // 2
+        total += 4 * d * pairs
+    return B * total
