@@ -1,0 +1,448 @@
+"""Benchmark of the MoA hot path on B200: heterogeneous sliding-window prefill and decode.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * span rule for the prompt (host), Vicuna-7B-shaped bf16 prefill
+    (B=1, 32 heads, d=128, N=8192, spans rescaled to mean span/N = 25%) with
+    the prompt's K/V appended to a per-head ring cache;
+  * one Vicuna-7B-shaped decode step: 32 layers x (append the new token's K/V,
+    decode attention) for B=32 sequences, 32 heads, d=128, context 4096,
+    per-layer elastic spans at 50% mean density, caches prefilled with N(0,1).
+
+The JSON line reports decode attention tokens/s (the headline ``value``), KV
+GB/s, prefill in-window TFLOP/s, each with its roofline fraction, the oracle
+timed on the host cores beside it, an end-to-end number through the C ABI
+with host buffers, and the SM clocks sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own replica (batch-sharded decode, its own
+prompt: weak scaling, no collective on the data path); timings are the max
+over ranks.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attn tokens/s + KV HBM GB/s; prefill in-window TFLOP/s (% of roofline)"
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+# workload
+P_B, P_H, P_N, P_D, P_DENSITY, P_SEED = 1, 32, 8192, 128, 0.25, 1
+D_L, D_B, D_H, D_N, D_D, D_DENSITY, D_SEED = 32, 32, 32, 4096, 128, 0.5, 1000
+BLOCK = 64
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _workload_desc():
+    return ("vicuna7b-shaped: prefill B=%d H=%d d=%d N=%d density %.2f + decode %dL x %dH B=%d d=%d ctx %d "
+            "density %.2f" % (P_B, P_H, P_D, P_N, P_DENSITY, D_L, D_H, D_B, D_D, D_N, D_DENSITY))
+
+
+def _config():
+    return {"workload": _workload_desc(), "prefill_shape": [P_B, P_H, P_N, P_D], "decode_shape":
+            [D_L, D_B, D_H, D_N, D_D], "block": BLOCK, "seeds": {"prefill": P_SEED, "decode": D_SEED},
+            "l2": "inputs larger than L2 (decode reads ~34 GB/step; prefill Q/K/V 192 MiB)",
+            "parallelism": "replica per GPU (batch-sharded decode, one prompt per GPU)"}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        finally:
+            os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline, never the product path)
+# ---------------------------------------------------------------------------
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_decode_sample(seconds_budget=10.0, seqs=2):
+    """Oracle decode tokens/s on a bounded sample: `seqs` sequences x 32 heads x 32 layers."""
+    from oracle import attention as oatt, rules as orules
+    from heterogeneous_sliding_window_b200 import inputs
+    rng = np.random.default_rng(7)
+    scale = 1.0 / math.sqrt(D_D)
+    timed = 0.0
+    rows = 0
+    layers_done = 0
+    for layer in range(D_L):
+        a, b = inputs.tables_7b(D_SEED + layer, D_H, D_N, BLOCK, D_DENSITY, orules.eval_spans)
+        spans = orules.eval_spans(a, b, D_N, BLOCK)
+        for _ in range(seqs):
+            for h in range(D_H):
+                S = spans[h]
+                K = rng.standard_normal((S, D_D))
+                V = rng.standard_normal((S, D_D))
+                q = rng.standard_normal(D_D)
+                t0 = time.perf_counter()
+                oatt.attend_row(q, K, V, 0, S - 1, scale)
+                timed += time.perf_counter() - t0
+                rows += 1
+        layers_done += 1
+        if timed > seconds_budget:
+            break
+    # tokens/s: one token = one sequence through all D_L layers
+    per_token = timed / (seqs * layers_done) * D_L
+    return 1.0 / per_token, "%d sequences x %d heads x %d of %d layers (fresh N(0,1) windows), per-token time " \
+        "extrapolated to %d layers" % (seqs, D_H, layers_done, D_L, D_L)
+
+
+def oracle_prefill_sample(seconds_budget=10.0):
+    """Oracle prefill GFLOP/s (in-window) on a bounded sample of query rows of the 7B prompt."""
+    from oracle import attention as oatt, rules as orules
+    from heterogeneous_sliding_window_b200 import inputs
+    a, b = inputs.tables_7b(P_SEED, P_H, P_N, BLOCK, P_DENSITY, orules.eval_spans)
+    spans = orules.eval_spans(a, b, P_N, BLOCK)
+    rng = np.random.default_rng(8)
+    K = rng.standard_normal((P_N, P_D))
+    V = rng.standard_normal((P_N, P_D))
+    scale = 1.0 / math.sqrt(P_D)
+    timed, flops, n = 0.0, 0, 0
+    for i in list(range(P_N - 1, 0, -97)):
+        for h in range(0, P_H, 4):
+            S = spans[h]
+            lo = max(0, i - S + 1)
+            q = rng.standard_normal(P_D)
+            t0 = time.perf_counter()
+            oatt.attend_row(q, K, V, lo, i, scale)
+            timed += time.perf_counter() - t0
+            flops += 4 * P_D * (i - lo + 1)
+            n += 1
+        if timed > seconds_budget:
+            break
+    return flops / timed / 1e9, "%d query rows (every 97th row x every 4th head) of the prompt" % n
+
+
+# ---------------------------------------------------------------------------
+# GPU path
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    from heterogeneous_sliding_window_b200 import build as _build
+
+    ws_n, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if not os.path.exists(moa.LIB_PATH):
+        _build.build()
+    moa.load()
+    dev = "cuda"
+    stream = torch.cuda.current_stream()
+    hbm_peak, tf_peak, tf_sustained, peak_kind = _peaks()
+
+    # ---- prefill inputs (rank-specific seeds: each rank its own prompt)
+    pa, pb = inputs.tables_7b(P_SEED, P_H, P_N, BLOCK, P_DENSITY, moa.moa_rules_eval)
+    p_spans = moa.moa_rules_eval(pa, pb, P_N, BLOCK)
+    q = inputs.randn_cuda(10 + 7 * rank, (P_B, P_H, P_N, P_D))
+    k = inputs.randn_cuda(11 + 7 * rank, (P_B, P_H, P_N, P_D))
+    v = inputs.randn_cuda(12 + 7 * rank, (P_B, P_H, P_N, P_D))
+    o = torch.empty_like(q)
+    p_scale = 1.0 / math.sqrt(P_D)
+    p_ws = moa.Workspace(moa.MOA_OP_PREFILL, P_B, P_H, P_N, P_D, p_spans)
+    p_cache = moa.KVCache(P_B, P_H, P_D, "bf16", p_spans)
+    p_flops = sum(4 * P_D * (min(S, P_N) * P_N - min(S, P_N) * (min(S, P_N) - 1) // 2) for S in p_spans) * P_B
+
+    # ---- decode state: 32 layers of caches prefilled with N(0,1), positions = context
+    d_spans, caches, d_ws, d_q, d_k, d_v, d_o = [], [], [], [], [], [], []
+    for layer in range(D_L):
+        a, b = inputs.tables_7b(D_SEED + layer, D_H, D_N, BLOCK, D_DENSITY, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, D_N, BLOCK)
+        d_spans.append(sp)
+        c = moa.KVCache(D_B, D_H, D_D, "bf16", sp)
+        data = c.data_bytes().view(torch.bfloat16)
+        data.copy_(inputs.randn_cuda(100 + layer + 1000 * rank, (data.numel(),)))
+        c.set_positions([D_N] * D_B)
+        caches.append(c)
+        d_ws.append(moa.Workspace(moa.MOA_OP_DECODE, D_B, D_H, 0, D_D, sp))
+        d_q.append(inputs.randn_cuda(200 + layer, (D_B, D_H, D_D)))
+        d_k.append(inputs.randn_cuda(300 + layer, (D_B, D_H, 1, D_D)))
+        d_v.append(inputs.randn_cuda(400 + layer, (D_B, D_H, 1, D_D)))
+        d_o.append(torch.empty((D_B, D_H, D_D), dtype=torch.bfloat16, device=dev))
+    torch.cuda.synchronize()
+    d_scale = 1.0 / math.sqrt(D_D)
+    kv_bytes_layer = [D_B * sum(2 * S * D_D * 2 for S in sp) + 2 * D_B * D_H * D_D * 2 for sp in d_spans]
+    kv_bytes_step = sum(kv_bytes_layer)
+    launches_per_step = 2 + 2 * D_L
+
+    def step(ev):
+        # rule evaluation for the prompt (host), prefill, cache fill, decode step
+        moa.moa_rules_eval(pa, pb, P_N, BLOCK)
+        ev["p0"].record(stream)
+        moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", p_spans, p_scale, p_ws.ptr, p_ws.nbytes,
+                        None, stream)
+        ev["p1"].record(stream)
+        moa.moa_kv_append(p_cache.handle, k, v, P_N, stream)
+        ev["d0"].record(stream)
+        for layer in range(D_L):
+            moa.moa_kv_append(caches[layer].handle, d_k[layer], d_v[layer], 1, stream)
+            ev["k0"][layer].record(stream)
+            moa.moa_decode(caches[layer].handle, d_q[layer], d_o[layer], D_H, d_spans[layer], d_scale,
+                           d_ws[layer].ptr, d_ws[layer].nbytes, stream)
+            ev["k1"][layer].record(stream)
+        ev["d1"].record(stream)
+
+    def new_events():
+        E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+        return {"p0": E(), "p1": E(), "d0": E(), "d1": E(), "k0": [E() for _ in range(D_L)],
+                "k1": [E() for _ in range(D_L)]}
+
+    for _ in range(args.warmup):
+        step(new_events())
+    torch.cuda.synchronize()
+    moa.moa_workspace_check(p_ws.ptr)
+
+    clocks = Clocks(torch.cuda.current_device())
+    evs = [new_events() for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = sum(e["p0"].elapsed_time(e["p1"]) for e in evs) / args.steps
+    decode_ms = sum(e["d0"].elapsed_time(e["d1"]) for e in evs) / args.steps
+    dec_kernel_ms = sum(e["k0"][l].elapsed_time(e["k1"][l]) for e in evs for l in range(D_L)) / (args.steps * D_L)
+    moa.moa_workspace_check(p_ws.ptr)
+    for c in caches:
+        c.positions()
+
+    vals = torch.tensor([total_ms, prefill_ms, decode_ms, dec_kernel_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, prefill_ms, decode_ms, dec_kernel_ms = vals.tolist()
+    ms_per_step = total_ms / args.steps
+
+    tokens_per_s = ws_n * D_B / (decode_ms * 1e-3)
+    kv_gbs = ws_n * kv_bytes_step / (decode_ms * 1e-3) / 1e9
+    prefill_tflops = ws_n * p_flops / (prefill_ms * 1e-3) / 1e12
+    dec_bytes_launch = sum(kv_bytes_layer) / D_L
+    dec_achieved = dec_bytes_launch / (dec_kernel_ms * 1e-3) / 1e9
+    p_achieved = p_flops / (prefill_ms * 1e-3) / 1e12
+
+    # ---- end to end through the C ABI with host buffers (pinned), decode step
+    h_q = [x.cpu().pin_memory() for x in d_q]
+    h_k = [x.cpu().pin_memory() for x in d_k]
+    h_v = [x.cpu().pin_memory() for x in d_v]
+    h_o = [torch.empty((D_B, D_H, D_D), dtype=torch.bfloat16).pin_memory() for _ in range(D_L)]
+    e_q = [torch.empty_like(x) for x in d_q]
+    e_k = [torch.empty_like(x) for x in d_k]
+    e_v = [torch.empty_like(x) for x in d_v]
+
+    def e2e_step():
+        for layer in range(D_L):
+            e_q[layer].copy_(h_q[layer], non_blocking=True)
+            e_k[layer].copy_(h_k[layer], non_blocking=True)
+            e_v[layer].copy_(h_v[layer], non_blocking=True)
+            moa.moa_kv_append(caches[layer].handle, e_k[layer], e_v[layer], 1, stream)
+            moa.moa_decode(caches[layer].handle, e_q[layer], d_o[layer], D_H, d_spans[layer], d_scale,
+                           d_ws[layer].ptr, d_ws[layer].nbytes, stream)
+            h_o[layer].copy_(d_o[layer], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = e2e_ms.item()
+    h2d = sum(x.numel() * x.element_size() for x in h_q + h_k + h_v)
+    d2h = sum(x.numel() * x.element_size() for x in h_o)
+
+    result = None
+    if rank == 0:
+        cpu_tok, cpu_sample = oracle_decode_sample(args.cpu_seconds)
+        cpu_gflops, cpu_p_sample = oracle_prefill_sample(args.cpu_seconds)
+        traffic = _ncu_traffic()
+        result = {
+            "metric": METRIC, "value": round(tokens_per_s, 2), "unit": "tokens/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Q/K/V and caches; Vicuna-7B-shaped; no weights or datasets)",
+            "config": _config(),
+            "kv_gbs": round(kv_gbs, 2),
+            "decode_ms_per_step": round(decode_ms, 4),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel<bf16,128> (moa_decode, one layer)",
+                         "achieved": round(dec_achieved, 2), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(dec_achieved / hbm_peak, 4), "peak_kind": peak_kind + " copy (hbm_gbs)",
+                         "frac_of_nominal": round(dec_achieved / NOMINAL_HBM_GBS, 4),
+                         "traffic": traffic.get("decode"),
+                         "algorithmic_bytes_per_launch": int(dec_bytes_launch)},
+            "prefill": {"tflops": round(prefill_tflops, 2), "ms": round(prefill_ms, 4),
+                        "spans": p_spans, "in_window_flops": int(p_flops),
+                        "roofline": {"bound": "tensor", "kernel": "prefill_bf16_sm100_kernel (moa_prefill)",
+                                     "achieved": round(p_achieved, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                                     "frac": round(p_achieved / tf_peak, 4),
+                                     "peak_kind": peak_kind + " burst (bf16_tflops)",
+                                     "frac_of_sustained": round(p_achieved / tf_sustained, 4),
+                                     "frac_of_nominal": round(p_achieved / NOMINAL_BF16_TFLOPS, 4),
+                                     "traffic": traffic.get("prefill")}},
+            "e2e": {"value": round(ws_n * D_B / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "note": "decode step through the C ABI from pinned host q/k/v to host o"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clock_info,
+            "cpu_baseline": {"value": round(cpu_tok, 4), "unit": "tokens/s", "cores": _oracle_threads(),
+                             "host_cpus": os.cpu_count(), "kind": "oracle", "sample": cpu_sample,
+                             "prefill_gflops": round(cpu_gflops, 4), "prefill_sample": cpu_p_sample},
+        }
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def _ncu_traffic():
+    """Per-launch DRAM bytes from the committed ncu summaries, if they match the current kernels."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
+def run_reference(args):
+    ws_n, rank, _ = _dist()
+    if rank != 0:
+        return None
+    times = []
+    sample = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        tok, sample = oracle_decode_sample(args.cpu_seconds / 2, seqs=1)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(tok)
+    value = statistics.median(times)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(),
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": _oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,236 @@
+// C ABI front end of libmoa: argument validation and dispatch to the kernels.
+// Every check that can fail does so here, on the host, before anything is
+// enqueued; the kernels assume validated arguments.
+#include <cstring>
+#include <new>
+
+#include "internal.h"
+
+namespace moa {
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+}  // namespace moa
+
+using namespace moa;
+
+static bool valid_d(int32_t d) { return d == 64 || d == 128; }
+static bool valid_dtype(moa_dtype t) { return t == MOA_F32 || t == MOA_BF16; }
+
+extern "C" const char* moa_status_string(moa_status s) {
+  switch (s) {
+    case MOA_OK: return "MOA_OK";
+    case MOA_ERR_INVALID_ARG: return "MOA_ERR_INVALID_ARG";
+    case MOA_ERR_CAPACITY: return "MOA_ERR_CAPACITY";
+    case MOA_ERR_WORKSPACE: return "MOA_ERR_WORKSPACE";
+    case MOA_ERR_UNSUPPORTED: return "MOA_ERR_UNSUPPORTED";
+    case MOA_ERR_CUDA: return "MOA_ERR_CUDA";
+    case MOA_ERR_TIMEOUT: return "MOA_ERR_TIMEOUT";
+  }
+  return "MOA_ERR_UNKNOWN";
+}
+
+extern "C" moa_status moa_kv_header_bytes(int32_t B, size_t* bytes_out) {
+  if (B < 1 || !bytes_out) return MOA_ERR_INVALID_ARG;
+  *bytes_out = header_bytes(B);
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_bytes(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
+                                   const int32_t* capacity, size_t* bytes_out) {
+  if (B < 1 || Hkv < 1 || Hkv > MOA_MAX_HEADS || !valid_d(d) || !valid_dtype(dtype) ||
+      !capacity || !bytes_out)
+    return MOA_ERR_INVALID_ARG;
+  int64_t sum = 0;
+  for (int32_t g = 0; g < Hkv; ++g) {
+    if (capacity[g] < 1) return MOA_ERR_INVALID_ARG;
+    sum += capacity[g];
+  }
+  *bytes_out = header_bytes(B) + (size_t)B * (size_t)sum * 2 * (size_t)d * elem_bytes(dtype);
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_alloc(void* dev_buf, size_t bytes, int32_t B, int32_t Hkv, int32_t d,
+                                   moa_dtype dtype, const int32_t* capacity, void* stream,
+                                   moa_kv_cache** out) {
+  if (!out) return MOA_ERR_INVALID_ARG;
+  *out = nullptr;
+  size_t need = 0;
+  moa_status st = moa_kv_bytes(B, Hkv, d, dtype, capacity, &need);
+  if (st != MOA_OK) return st;
+  if (!dev_buf || ((uintptr_t)dev_buf & 255u) != 0) return MOA_ERR_INVALID_ARG;
+  if (bytes < need) return MOA_ERR_CAPACITY;
+  moa_kv_cache* c = new (std::nothrow) moa_kv_cache();
+  if (!c) return MOA_ERR_INVALID_ARG;
+  c->buf = (char*)dev_buf;
+  c->bytes = need;
+  c->B = B;
+  c->Hkv = Hkv;
+  c->d = d;
+  c->dtype = dtype;
+  c->header = header_bytes(B);
+  c->cap.assign(capacity, capacity + Hkv);
+  c->goff.assign(Hkv + 1, 0);
+  for (int32_t g = 0; g < Hkv; ++g) c->goff[g + 1] = c->goff[g] + capacity[g];
+  if (cudaMemsetAsync(dev_buf, 0, need, (cudaStream_t)stream) != cudaSuccess) {
+    delete c;
+    return MOA_ERR_CUDA;
+  }
+  *out = c;
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_free(moa_kv_cache* cache) {
+  delete cache;
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_layout(const moa_kv_cache* c, void** data_out, int64_t* goff) {
+  if (!c || !data_out) return MOA_ERR_INVALID_ARG;
+  *data_out = c->buf + c->header;
+  if (goff)
+    for (int32_t g = 0; g <= c->Hkv; ++g) goff[g] = c->goff[g];
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
+                                    void* stream) {
+  if (!c || !k || !v || n_tok < 1) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return MOA_ERR_INVALID_ARG;
+  return launch_append(c, k, v, n_tok, (cudaStream_t)stream);
+}
+
+extern "C" moa_status moa_kv_positions(const moa_kv_cache* c, int64_t* t_host, void* stream) {
+  if (!c || !t_host) return MOA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t err = 0;
+  if (cudaMemcpyAsync(&err, c->buf + kHdrErr, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return MOA_ERR_CUDA;
+  if (cudaMemcpyAsync(t_host, c->buf + kHdrT, 8 * (size_t)c->B, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return MOA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOA_ERR_CUDA;
+  if (err & kErrTimeout) return MOA_ERR_TIMEOUT;
+  return err ? MOA_ERR_INVALID_ARG : MOA_OK;
+}
+
+extern "C" moa_status moa_kv_set_positions(moa_kv_cache* c, const int64_t* t_host, void* stream) {
+  if (!c || !t_host) return MOA_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < c->B; ++b)
+    if (t_host[b] < 0) return MOA_ERR_INVALID_ARG;
+  // Pageable source: the runtime stages it before returning, so t_host may be
+  // reused as soon as this call returns.
+  if (cudaMemcpyAsync(c->buf + kHdrT, t_host, 8 * (size_t)c->B, cudaMemcpyHostToDevice,
+                      (cudaStream_t)stream) != cudaSuccess)
+    return MOA_ERR_CUDA;
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_workspace_bytes(moa_op op, int32_t B, int32_t Hq, int64_t N, int32_t d,
+                                          const int32_t* spans, size_t* bytes_out) {
+  if (!bytes_out || B < 1 || Hq < 1 || Hq > MOA_MAX_HEADS || !valid_d(d)) return MOA_ERR_INVALID_ARG;
+  if (op == MOA_OP_PREFILL) {
+    if (N < 1 || N > INT32_MAX) return MOA_ERR_INVALID_ARG;
+    *bytes_out = prefill_workspace_bytes(B, Hq, N);
+    return MOA_OK;
+  }
+  if (op == MOA_OP_DECODE) {
+    if (!spans) return MOA_ERR_INVALID_ARG;
+    for (int32_t h = 0; h < Hq; ++h)
+      if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+    *bytes_out = decode_workspace_bytes(B, Hq, d, spans);
+    return MOA_OK;
+  }
+  return MOA_ERR_INVALID_ARG;
+}
+
+extern "C" moa_status moa_workspace_init(void* ws, size_t bytes, void* stream) {
+  if (!ws || bytes == 0) return MOA_ERR_INVALID_ARG;
+  return cudaMemsetAsync(ws, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
+}
+
+extern "C" moa_status moa_workspace_check(const void* ws, void* stream) {
+  if (!ws) return MOA_ERR_INVALID_ARG;
+  uint32_t err = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&err, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOA_ERR_CUDA;
+  return err ? MOA_ERR_TIMEOUT : MOA_OK;
+}
+
+extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
+                                           int32_t* units_out, int64_t cap, int64_t* n_units_out) {
+  if (B < 1 || Hq < 1 || Hq > MOA_MAX_HEADS || N < 1 || N > INT32_MAX || !spans || !n_units_out ||
+      cap < 0 || (cap > 0 && !units_out))
+    return MOA_ERR_INVALID_ARG;
+  for (int32_t h = 0; h < Hq; ++h)
+    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+  std::vector<int32_t> u = prefill_units(B, Hq, (int32_t)N, spans);
+  const int64_t n = (int64_t)u.size() / 4;
+  *n_units_out = n;
+  for (int64_t i = 0; i < n && i < cap; ++i) {
+    units_out[5 * i + 0] = u[4 * i + 0];
+    units_out[5 * i + 1] = u[4 * i + 1];
+    units_out[5 * i + 2] = u[4 * i + 2];
+    units_out[5 * i + 3] = u[4 * i + 3];
+    units_out[5 * i + 4] = u[4 * i + 2];  // hi: the diagonal tile
+  }
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, void* o, int32_t B,
+                                  int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
+                                  const int32_t* spans, float scale, void* ws, size_t ws_bytes,
+                                  moa_kv_cache* fill, void* stream) {
+  if (!q || !k || !v || !o || !spans) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq > MOA_MAX_HEADS || Hkv > MOA_MAX_HEADS || Hq % Hkv != 0)
+    return MOA_ERR_INVALID_ARG;
+  if (N < 1 || N > INT32_MAX || !valid_d(d) || !valid_dtype(dtype)) return MOA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
+  for (int32_t h = 0; h < Hq; ++h)
+    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+  const int32_t G = Hq / Hkv;
+  if (fill) {
+    if (fill->B != B || fill->Hkv != Hkv || fill->d != d || fill->dtype != dtype)
+      return MOA_ERR_INVALID_ARG;
+    for (int32_t h = 0; h < Hq; ++h)
+      if (spans[h] > fill->cap[h / G]) return MOA_ERR_CAPACITY;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  moa_status st;
+  if (dtype == MOA_F32) {
+    st = launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (float*)o, B, Hq, Hkv,
+                            (int32_t)N, d, spans, scale, s);
+  } else {
+    if (d != 128) return MOA_ERR_UNSUPPORTED;
+    if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
+    if (ws_bytes < prefill_workspace_bytes(B, Hq, N)) return MOA_ERR_WORKSPACE;
+    st = launch_prefill_bf16(q, k, v, o, B, Hq, Hkv, (int32_t)N, spans, scale, ws, ws_bytes, s);
+  }
+  if (st != MOA_OK || !fill) return st;
+  return launch_append(fill, k, v, (int32_t)N, s);
+}
+
+extern "C" moa_status moa_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
+                                 const int32_t* spans, float scale, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!c || !q || !o || !spans) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if (Hq < 1 || Hq > MOA_MAX_HEADS || Hq % c->Hkv != 0) return MOA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
+  const int32_t G = Hq / c->Hkv;
+  for (int32_t h = 0; h < Hq; ++h) {
+    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+    if (spans[h] > c->cap[h / G]) return MOA_ERR_CAPACITY;
+  }
+  if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
+  if (ws_bytes < decode_workspace_bytes(c->B, Hq, c->d, spans)) return MOA_ERR_WORKSPACE;
+  return launch_decode(c, q, o, Hq, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
+}

@@ -1,0 +1,67 @@
+// Internal declarations shared by the translation units of libmoa.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include <vector>
+
+#include "moa.h"
+
+#define MOA_MAX_HEADS 128
+
+struct moa_kv_cache {
+  char* buf = nullptr;           // caller-owned device buffer
+  size_t bytes = 0;
+  int32_t B = 0, Hkv = 0, d = 0;
+  moa_dtype dtype = MOA_BF16;
+  size_t header = 0;             // bytes before the data region
+  std::vector<int32_t> cap;      // C_g
+  std::vector<int64_t> goff;     // prefix sums of C_g, size Hkv + 1
+};
+
+namespace moa {
+
+inline size_t elem_bytes(moa_dtype t) { return t == MOA_F32 ? 4 : 2; }
+inline size_t header_bytes(int64_t B) { return (size_t)(((16 + 8 * B) + 255) / 256 * 256); }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Header field offsets (bytes) inside a cache buffer.
+constexpr size_t kHdrErr = 0;
+constexpr size_t kHdrAppendCtr = 4;
+constexpr size_t kHdrT = 16;
+
+// Device error bits (cache and workspace error words).
+constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrEmpty = 2u;
+
+int sm_count();
+
+// kv.cu
+moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
+                         cudaStream_t s);
+
+// decode.cu
+size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans);
+moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
+                         const int32_t* spans, float scale, void* ws, size_t ws_bytes,
+                         cudaStream_t s);
+
+// prefill_simt.cu (fp32)
+moa_status launch_prefill_f32(const float* q, const float* k, const float* v, float* o,
+                              int32_t B, int32_t Hq, int32_t Hkv, int32_t N, int32_t d,
+                              const int32_t* spans, float scale, cudaStream_t s);
+
+// prefill_sm100.cu (bf16, tcgen05)
+constexpr int kTileM = 128;   // query rows per work unit
+constexpr int kTileN = 128;   // keys per key/value tile
+struct Unit { int32_t b, h, m, lo; };     // key tiles lo..m (the diagonal tile is m)
+std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans);
+size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
+moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,
+                               int32_t B, int32_t Hq, int32_t Hkv, int32_t N,
+                               const int32_t* spans, float scale, void* ws, size_t ws_bytes,
+                               cudaStream_t s);
+
+}  // namespace moa

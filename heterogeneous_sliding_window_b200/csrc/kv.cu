@@ -1,0 +1,96 @@
+// Per-head ring-buffer KV cache: append kernel.
+//
+// "Mixture of Attention" project page, "Demo" step 03: decoding is served
+// from a fixed-size KV cache sized per head.  Token position p of a sequence
+// is kept in slot p mod C_g of its key/value head g, so the buffer always
+// holds the last C_g tokens -- all that a head with span S_h <= C_g reads.
+#include "internal.h"
+
+namespace moa {
+namespace {
+
+constexpr int kAppendRows = 64;      // rows per block and per key/value head
+constexpr int kAppendThreads = 256;
+
+struct AppendParams {
+  char* data;                 // data region of the cache buffer
+  uint32_t* ctr;              // header: completion counter
+  int64_t* t;                 // header: tokens per sequence
+  const char* k;
+  const char* v;
+  int32_t Hkv, n_tok, row_bytes;
+  int64_t sumC;
+  int32_t cap[MOA_MAX_HEADS];
+  int64_t goff[MOA_MAX_HEADS];
+};
+
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(const __grid_constant__ AppendParams p) {
+  const int g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int C = p.cap[g];
+  const int nrows = p.n_tok < C ? p.n_tok : C;   // only the last C rows survive
+  const int r0 = blockIdx.x * kAppendRows;
+  const int64_t t0 = p.t[b];
+  if (r0 < nrows) {
+    const int rows = min(kAppendRows, nrows - r0);
+    const int vpr = p.row_bytes / 16;
+    const int first = p.n_tok - nrows;          // source row of the first survivor
+    char* kdst = p.data + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * p.row_bytes;
+    char* vdst = kdst + (size_t)C * p.row_bytes;
+    const size_t src_base = ((size_t)b * p.Hkv + g) * (size_t)p.n_tok;
+    for (int idx = threadIdx.x; idx < rows * vpr; idx += kAppendThreads) {
+      const int rr = idx / vpr;
+      const int vv = idx - rr * vpr;
+      const int r = first + r0 + rr;
+      const int64_t slot = (t0 + r) % C;
+      const size_t src = (src_base + r) * p.row_bytes + (size_t)vv * 16;
+      const size_t dst = (size_t)slot * p.row_bytes + (size_t)vv * 16;
+      const int4 kv = __ldg(reinterpret_cast<const int4*>(p.k + src));
+      const int4 vv4 = __ldg(reinterpret_cast<const int4*>(p.v + src));
+      *reinterpret_cast<int4*>(kdst + dst) = kv;
+      *reinterpret_cast<int4*>(vdst + dst) = vv4;
+    }
+  }
+  // The last block to finish advances every sequence's position.  All blocks
+  // read t[b] above, before they take a ticket, so none sees the new value.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned total = gridDim.x * gridDim.y * gridDim.z;
+    const unsigned prev = atomicAdd(p.ctr, 1u);
+    if (prev == total - 1) {
+      const int B = gridDim.z;
+      for (int bb = 0; bb < B; ++bb) p.t[bb] += p.n_tok;
+      *p.ctr = 0u;
+      __threadfence();
+    }
+  }
+}
+
+}  // namespace
+
+moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
+                         cudaStream_t s) {
+  AppendParams p;
+  p.data = c->buf + c->header;
+  p.ctr = reinterpret_cast<uint32_t*>(c->buf + kHdrAppendCtr);
+  p.t = reinterpret_cast<int64_t*>(c->buf + kHdrT);
+  p.k = (const char*)k;
+  p.v = (const char*)v;
+  p.Hkv = c->Hkv;
+  p.n_tok = n_tok;
+  p.row_bytes = c->d * (int)elem_bytes(c->dtype);
+  p.sumC = c->goff[c->Hkv];
+  int maxrows = 0;
+  for (int g = 0; g < c->Hkv; ++g) {
+    p.cap[g] = c->cap[g];
+    p.goff[g] = c->goff[g];
+    const int r = n_tok < c->cap[g] ? n_tok : c->cap[g];
+    if (r > maxrows) maxrows = r;
+  }
+  dim3 grid((maxrows + kAppendRows - 1) / kAppendRows, c->Hkv, c->B);
+  append_kernel<<<grid, kAppendThreads, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
+}
+
+}  // namespace moa

@@ -1,0 +1,196 @@
+/*
+ * moa.h -- C ABI of libmoa: heterogeneous sliding-window attention (MoA) on B200.
+ *
+ * The method ("Mixture of Attention" project page, section "Key findings /
+ * Finding two: windows change with input length") gives every attention head
+ * h its own causal sliding window whose length follows a linear rule in the
+ * input length N, S_h = alpha_h + beta_h * N.  Query row i of head h attends
+ * only to keys j with i - S_h < j <= i.  Deployment ("Demo", step 03, same
+ * page) serves decoding from a fixed-size KV cache whose size differs per
+ * head; the blog walkthrough "MoA: Mixture of Sparse Attention for Automatic
+ * Large Language Model Compression", section 5, implements the static KV
+ * cache, the mask and the attention aggregation in a CUDA kernel.
+ *
+ * Conventions for every entry point
+ *  - Device pointers are plain CUDA device addresses owned by the caller; the
+ *    library never allocates or frees device memory.  Host pointers are read
+ *    (or written) before the call returns unless stated otherwise.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Device work is enqueued asynchronously on it; the caller keeps every
+ *    buffer alive until that work has completed.
+ *  - Argument errors are detected on the host, return a status and launch
+ *    nothing.  Launch failures return MOA_ERR_CUDA.  Nothing calls exit/abort.
+ *  - Tensors are dense, row-major, 16-byte aligned:
+ *      q, o : [B, Hq,  N, d]     k, v : [B, Hkv, N, d]     (prefill)
+ *      q, o : [B, Hq,  d]        k, v : [B, Hkv, n_tok, d] (decode / append)
+ *    with grouped-query attention: query head h reads key/value head h / (Hq/Hkv).
+ *  - Supported: d in {64, 128}; dtype MOA_F32 for d 64/128 (SIMT, fp32
+ *    throughout); dtype MOA_BF16 for d 128 (tensor cores, fp32 accumulate).
+ *    Hq <= 128, Hkv <= 128, Hq % Hkv == 0, 1 <= N < 2^31, B >= 1.
+ */
+#ifndef MOA_H
+#define MOA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOA_OK = 0,
+  MOA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or shape, NaN rule */
+  MOA_ERR_CAPACITY = 2,     /* a span exceeds its key/value head's cache capacity  */
+  MOA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moa_workspace_bytes */
+  MOA_ERR_UNSUPPORTED = 4,  /* valid request this build does not implement (e.g. bf16 d=64) */
+  MOA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+  MOA_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (error word set) */
+} moa_status;
+
+typedef enum { MOA_F32 = 0, MOA_BF16 = 1 } moa_dtype;
+
+typedef enum { MOA_OP_PREFILL = 0, MOA_OP_DECODE = 1 } moa_op;
+
+/* Opaque host-side handle describing a caller-owned cache buffer. */
+typedef struct moa_kv_cache moa_kv_cache;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moa_status_string(moa_status s);
+
+/* ---------------------------------------------------------------------------
+ * Span rule.  "Mixture of Attention" project page, "Finding two" (S = alpha +
+ * beta * N), "Method design / Elastic search space" (spans respect the
+ * kernel's block size) and the heads A/B/C panel (span clamped to N).
+ *   x = alpha[h] + beta[h] * (double)N      (binary64, two separate roundings)
+ *   S = block * floor(x / block + 0.5)      (nearest multiple, ties up)
+ *   spans_out[h] = min(N, max(block, S))
+ * Host only; no CUDA call.  alpha/beta must be finite and >= 0, N >= 1,
+ * 1 <= block, n_heads >= 1.  Writes n_heads int32 values.  Spans above
+ * INT32_MAX cannot occur because N < 2^31 is required.
+ * ------------------------------------------------------------------------- */
+moa_status moa_rules_eval(const double* alpha, const double* beta, int32_t n_heads,
+                          int64_t N, int32_t block, int32_t* spans_out);
+
+/* ---------------------------------------------------------------------------
+ * Per-head ring-buffer KV cache ("Demo" step 03: fixed-size per-head cache).
+ * Key/value head g of each sequence owns C_g = capacity[g] slots; token
+ * position p lives in slot p mod C_g, so the ring always holds the last C_g
+ * tokens, which serve every query head of the group whose span is <= C_g.
+ *
+ * Buffer layout (caller-owned device memory, size from moa_kv_bytes):
+ *   header, H = round_up(16 + 8*B, 256) bytes:
+ *     bytes 0..3   uint32 error word (0 = ok; bit 0 = bounded wait timed out,
+ *                  bit 1 = decode found an empty sequence)
+ *     bytes 4..7   uint32 append-completion counter (internal, returns to 0)
+ *     bytes 8..15  reserved, zero
+ *     bytes 16..   int64 t[B]: tokens appended so far, per sequence
+ *   data at byte H: for b in [0,B), for g in [0,Hkv): K block [C_g][d], then
+ *     V block [C_g][d], elements of the cache dtype.  The K block of (b, g)
+ *     starts at element (b * sum_g C_g + sum_{g'<g} C_g') * 2 * d.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of the buffer for the layout above.  capacity: host int32[Hkv], >= 1. */
+moa_status moa_kv_bytes(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
+                        const int32_t* capacity, size_t* bytes_out);
+
+/* Size of the header region (the data region starts at this byte offset). */
+moa_status moa_kv_header_bytes(int32_t B, size_t* bytes_out);
+
+/* Bind a caller-owned device buffer of at least moa_kv_bytes bytes (256-byte
+ * aligned) as an empty cache: zeroes the whole buffer on `stream` and returns a
+ * new host handle in *out.  The handle copies `capacity`; it never owns
+ * dev_buf.  Release the handle with moa_kv_free. */
+moa_status moa_kv_alloc(void* dev_buf, size_t bytes, int32_t B, int32_t Hkv, int32_t d,
+                        moa_dtype dtype, const int32_t* capacity, void* stream,
+                        moa_kv_cache** out);
+
+/* Free the host handle (not the device buffer).  NULL is accepted. */
+moa_status moa_kv_free(moa_kv_cache* cache);
+
+/* Append n_tok >= 1 tokens per sequence.  k, v: device [B, Hkv, n_tok, d] in
+ * the cache dtype.  Token r of sequence b gets position t_b + r and is stored
+ * in slot (t_b + r) mod C_g; only the last min(n_tok, C_g) rows are copied,
+ * the rest would be overwritten.  Then t_b += n_tok (on the device, in the
+ * same launch).  Calls on one cache must be ordered on one stream. */
+moa_status moa_kv_append(moa_kv_cache* cache, const void* k, const void* v,
+                         int32_t n_tok, void* stream);
+
+/* Read t[B] into host memory t_host and check the error word.  Synchronises
+ * `stream`.  Returns MOA_ERR_TIMEOUT if error bit 0 is set, MOA_ERR_INVALID_ARG
+ * if only bit 1 is (a decode ran on a sequence with no cached token), else
+ * MOA_OK.  The error word is sticky: clear it by re-binding the buffer. */
+moa_status moa_kv_positions(const moa_kv_cache* cache, int64_t* t_host, void* stream);
+
+/* Overwrite t[B] from host memory (e.g. restoring a cache whose data bytes the
+ * caller saved and copied back).  Enqueued on `stream`; t_host is consumed
+ * before return.  Every t_host[b] must be >= 0. */
+moa_status moa_kv_set_positions(moa_kv_cache* cache, const int64_t* t_host, void* stream);
+
+/* Device address of the data region and the slot offset of each key/value
+ * head: group_row_offset[g] = sum_{g'<g} C_g' for g in [0, Hkv], so
+ * group_row_offset[Hkv] = sum_g C_g.  group_row_offset may be NULL. */
+moa_status moa_kv_layout(const moa_kv_cache* cache, void** data_out, int64_t* group_row_offset);
+
+/* ---------------------------------------------------------------------------
+ * Workspace.  Caller-owned device scratch, 256-byte aligned.  A decode
+ * workspace must be zeroed once before its first use (moa_workspace_init or a
+ * memset); moa_decode leaves its counters at zero again.  A prefill workspace
+ * needs no initialisation.  Word 0 of every workspace is an error word.
+ * `spans` is host int32[Hq]; N is ignored for MOA_OP_DECODE.
+ * ------------------------------------------------------------------------- */
+moa_status moa_workspace_bytes(moa_op op, int32_t B, int32_t Hq, int64_t N, int32_t d,
+                               const int32_t* spans, size_t* bytes_out);
+
+/* Zero `bytes` bytes of workspace on `stream`. */
+moa_status moa_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/* Synchronise `stream` and read the workspace error word: MOA_ERR_TIMEOUT if a
+ * bounded wait in the last prefill using it gave up, else MOA_OK. */
+moa_status moa_workspace_check(const void* workspace, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Prefill: windowed causal attention over a whole prompt ("Finding two" and
+ * its N x N causal-band figure; blog section 2.1).  For every (b, h, i):
+ *   o[b,h,i,:] = softmax_j(scale * q[b,h,i,:] . k[b,g,j,:]) v[b,g,j,:]
+ * over j in (i - S_h, i], g = h / (Hq/Hkv).  spans: host int32[Hq], each >= 1
+ * (a span above N behaves as N).  MOA_BF16 runs the tensor-core kernel (d must
+ * be 128) and needs a workspace of moa_workspace_bytes(MOA_OP_PREFILL, ...)
+ * bytes; MOA_F32 may pass workspace NULL.  The schedule of work units is
+ * uploaded into the workspace from host memory on every call.
+ * fill_or_null: if non-NULL, a cache with B, Hkv, d and dtype equal to this
+ * call's, spans[h] <= C_{h/(Hq/Hkv)}; after attention the prompt's K/V are
+ * appended to it exactly as moa_kv_append(cache, k, v, N) would.
+ * ------------------------------------------------------------------------- */
+moa_status moa_prefill(const void* q, const void* k, const void* v, void* o,
+                       int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
+                       moa_dtype dtype, const int32_t* spans, float scale,
+                       void* workspace, size_t ws_bytes, moa_kv_cache* fill_or_null,
+                       void* stream);
+
+/* Host view of the prefill schedule: one row of 5 int32 (b, h, m, lo, hi) per
+ * work unit -- query rows [128m, 128m+127] of head h, sequence b, visiting key
+ * tiles lo..hi of 128 keys -- in the order the persistent kernel takes them
+ * (longest first).  Writes min(cap, n) rows, *n_units_out = n.  Host only. */
+moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
+                                int32_t* units_out, int64_t cap, int64_t* n_units_out);
+
+/* ---------------------------------------------------------------------------
+ * Decode: one new query token per sequence against the ring cache.  Call
+ * moa_kv_append for the token's k, v first; then query head h of sequence b
+ * (at position t_b - 1) attends to positions j in (t_b - 1 - S_h, t_b - 1],
+ * read from slots j mod C_g.  q, o: device [B, Hq, d] in the cache dtype.
+ * spans: host int32[Hq], 1 <= spans[h] <= C_{h/(Hq/Hkv)}, else MOA_ERR_CAPACITY.
+ * workspace: moa_workspace_bytes(MOA_OP_DECODE, ...) bytes, zeroed before
+ * first use.  One kernel launch: split-KV partials with the log-sum-exp
+ * combine done by the last split of each (b, h).
+ * ------------------------------------------------------------------------- */
+moa_status moa_decode(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
+                      const int32_t* spans, float scale, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOA_H */

@@ -165,3 +165,36 @@ def data_image(cache, dtype):
             parts.append(_to_bits(cache.K[b][g], dtype))
             parts.append(_to_bits(cache.V[b][g], dtype))
     return b"".join(parts)
+
+
+def block_from_image(data, b, g, B, Hkv, d, capacities, dtype):
+    """K and V rows [C_g, d] of (sequence b, kv head g) read from a data-region image.
+
+    ``data`` is a bytes-like image of the data region laid out as documented
+    above; returns float64 arrays in slot order.
+    """
+    eb = 4 if dtype == "f32" else 2
+    sumC = sum(int(c) for c in capacities)
+    C = int(capacities[g])
+    start = (b * sumC + sum(int(c) for c in capacities[:g])) * 2 * d
+    raw = np.frombuffer(bytes(data[start * eb:(start + 2 * C * d) * eb]),
+                        dtype="<u4" if eb == 4 else "<u2")
+    if eb == 4:
+        vals = raw.view("<f4").astype(np.float64)
+    else:
+        vals = (raw.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    vals = vals.reshape(2, C, d)
+    return vals[0].copy(), vals[1].copy()
+
+
+def decode_row_from_ring(K, V, t, S, q, scale):
+    """Decode output of one (b, h) whose ring (slot order) is K, V after t tokens.
+
+    Attends to positions max(0, t - S) .. t - 1, each read from slot p mod C.
+    """
+    C = K.shape[0]
+    if S > C:
+        raise ValueError("span exceeds capacity")
+    pos = list(range(max(0, t - S), t))
+    idx = [p % C for p in pos]
+    return attend_row(q, K[idx], V[idx], 0, len(idx) - 1, scale)

@@ -1,0 +1,180 @@
+"""Host-side checks of libmoa's C ABI: symbols, span rule, schedule, sizes, argument errors.
+
+No test here launches a kernel; each runs without a GPU.
+"""
+
+import ctypes
+import os
+import random
+import re
+
+import numpy as np
+import pytest
+
+from heterogeneous_sliding_window_b200 import moa
+from heterogeneous_sliding_window_b200 import inputs
+from oracle import rules as orules, kvcache as okv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not os.path.exists(moa.LIB_PATH):
+        from heterogeneous_sliding_window_b200 import build
+        build.build()
+    moa.load()
+
+
+def _declared_symbols():
+    names = set()
+    with open(os.path.join(ROOT, "include", "moa.h")) as f:
+        text = f.read()
+    for m in re.finditer(r"^\s*(?:const\s+)?[\w\s\*]+?\b(moa_\w+)\s*\(", text, re.M):
+        names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_symbols()
+    assert len(declared) >= 15, declared
+    lib = ctypes.CDLL(moa.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    assert declared == set(moa.EXPORTS)
+
+
+def test_rules_bit_exact_against_oracle():
+    """10^6 random (alpha, beta, N, block) tuples, exact ties included."""
+    rnd = np.random.default_rng(11)
+    n_done = 0
+    while n_done < 1_000_000:
+        N = int(rnd.integers(1, 1 << 20))
+        block = int(rnd.choice([1, 16, 32, 64, 128, 256]))
+        n = 1000
+        kind = rnd.integers(0, 3)
+        if kind == 0:      # arbitrary doubles
+            a = rnd.uniform(0, 3 * N, n)
+            b = rnd.uniform(0, 1.5, n)
+        elif kind == 1:    # exact ties: alpha = (k + 1/2) * block, beta = 0
+            a = (rnd.integers(0, 2 * N // block + 2, n) + 0.5) * block
+            b = np.zeros(n)
+        else:              # candidate-set-like values
+            a = rnd.choice([0.0, 512.0, 1024.0, 2048.0, 1600.0, 5600.0], n) * rnd.choice([1.0, 0.37, 1.91], n)
+            b = rnd.choice([0.0, 0.125, 0.25, 0.5, 0.9, 1.0], n) * rnd.choice([1.0, 0.37, 1.91], n)
+        got = moa.moa_rules_eval(a, b, N, block)
+        ref = [orules.span_rule(x, y, N, block) for x, y in zip(a.tolist(), b.tolist())]
+        assert got == ref, (N, block)
+        n_done += n
+
+
+def test_rules_project_page_heads():
+    assert moa.moa_rules_eval([1600, 5600, 0], [0, 0, 0.9], 4096, 64) == [1600, 4096, 3712]
+    assert moa.moa_rules_eval([1600, 5600, 0], [0, 0, 0.9], 16384, 64) == [1600, 5632, 14720]
+
+
+@pytest.mark.parametrize("a,b,N,blk", [
+    (float("nan"), 0.0, 10, 1), (0.0, float("inf"), 10, 1), (-1.0, 0.0, 10, 1),
+    (1.0, 0.0, 0, 1), (1.0, 0.0, 10, 0), (1.0, 0.0, 1 << 31, 1)])
+def test_rules_invalid(a, b, N, blk):
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_rules_eval([a], [b], N, blk)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+
+
+def _tiles_needed_brute(m, S, N):
+    """Key tiles that hold at least one in-window key of some row of q-tile m."""
+    need = set()
+    for i in range(128 * m, min(128 * m + 128, N)):
+        for j in range(max(0, i - S + 1), i + 1):
+            need.add(j // 128)
+    return need
+
+
+@pytest.mark.parametrize("N,spans", [(1000, [1, 64, 127, 128, 129, 300, 1000, 5000]), (128, [1, 128]),
+                                     (129, [2, 129]), (5, [3])])
+def test_prefill_schedule_covers_band(N, spans):
+    B = 2
+    Hq = len(spans)
+    units = moa.moa_prefill_schedule(B, Hq, N, spans)
+    M = (N + 127) // 128
+    assert units.shape == (B * Hq * M, 5)
+    seen = set()
+    costs = []
+    for b, h, m, lo, hi in units.tolist():
+        assert (b, h, m) not in seen
+        seen.add((b, h, m))
+        assert hi == m
+        need = _tiles_needed_brute(m, spans[h], N)
+        assert set(range(lo, hi + 1)) == need   # exactly the band's tiles, none skipped, none extra
+        costs.append(hi - lo + 1)
+    assert len(seen) == B * Hq * M
+    assert costs == sorted(costs, reverse=True)  # longest first
+
+
+def test_kv_sizes_match_layout():
+    for B, Hkv, d, caps, dt, eb in [(2, 2, 4 * 16, [2, 3], "bf16", 2), (31, 3, 128, [5, 1, 9], "f32", 4),
+                                   (32, 32, 128, [2048] * 32, "bf16", 2)]:
+        assert moa.moa_kv_header_bytes(B) == okv.header_bytes(B)
+        assert moa.moa_kv_bytes(B, Hkv, d, dt, caps) == okv.buffer_bytes(B, Hkv, d, caps, eb)
+
+
+def test_kv_invalid():
+    with pytest.raises(moa.MoaError):
+        moa.moa_kv_bytes(1, 1, 96, "bf16", [4])       # head dim not supported
+    with pytest.raises(moa.MoaError):
+        moa.moa_kv_bytes(1, 2, 128, "bf16", [4, 0])   # zero capacity
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_kv_alloc(256, 10, 1, 1, 128, "bf16", [4])  # buffer too small
+    assert e.value.status == moa.MOA_ERR_CAPACITY
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_kv_alloc(8, 1 << 20, 1, 1, 128, "bf16", [4])  # misaligned
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+
+
+def test_prefill_argument_errors_need_no_gpu():
+    ok = dict(q=4096, k=4096, v=4096, o=4096, B=1, Hq=4, Hkv=2, N=256, d=128, dtype="bf16",
+              spans=[64] * 4, scale=0.088, ws=None, ws_bytes=0, stream=0)
+    bad = [dict(q=None), dict(q=4097), dict(Hq=3), dict(N=0), dict(d=96), dict(spans=[0, 1, 1, 1]),
+           dict(scale=float("nan"))]
+    for change in bad:
+        args = dict(ok)
+        args.update(change)
+        with pytest.raises(moa.MoaError) as e:
+            moa.moa_prefill(**args)
+        assert e.value.status == moa.MOA_ERR_INVALID_ARG, change
+    args = dict(ok)
+    with pytest.raises(moa.MoaError) as e:      # bf16 needs a workspace
+        moa.moa_prefill(**args)
+    assert e.value.status == moa.MOA_ERR_WORKSPACE
+    args.update(d=64, ws=4096, ws_bytes=1 << 20)
+    with pytest.raises(moa.MoaError) as e:      # bf16 d=64 not implemented
+        moa.moa_prefill(**args)
+    assert e.value.status == moa.MOA_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes():
+    spans = [64, 300, 4096, 1]
+    d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)
+    p = moa.moa_workspace_bytes(moa.MOA_OP_PREFILL, 2, 4, 1000, 128, spans)
+    assert d % 256 == 0 and d >= 256 + 2 * 4 * 4
+    assert p >= 256 + 2 * 4 * 8 * 16
+    with pytest.raises(moa.MoaError):
+        moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, [64, 0, 1, 1])
+
+
+def test_input_tables_reach_target_density():
+    """The seeded table generator lands near the requested mean span / N."""
+    for density, N in [(0.25, 8192), (0.5, 4096), (0.125, 32768)]:
+        a, b = inputs.tables_7b(3, 32, N, 64, density, orules.eval_spans)
+        spans = orules.eval_spans(a, b, N, 64)
+        assert abs(np.mean(spans) / N - density) < 0.02
+        assert all(s % 64 == 0 for s in spans)
+        # the product-side rule gives the same tables and spans
+        a2, b2 = inputs.tables_7b(3, 32, N, 64, density, moa.moa_rules_eval)
+        assert np.array_equal(a, a2) and np.array_equal(b, b2)
+        assert moa.moa_rules_eval(a2, b2, N, 64) == spans
+    a, b = inputs.tables_13b_mix(5, 40, 16384, 64, 0.5, orules.eval_spans)
+    spans = orules.eval_spans(a, b, 16384, 64)
+    assert abs(np.mean(spans) / 16384 - 0.5) < 0.05
+    assert set(np.unique(b)) <= {0.0, 0.5, 0.9}

@@ -1,0 +1,283 @@
+"""GPU parity: libmoa's kernels (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances: bf16 inputs with fp32 accumulation, max-abs 2e-2 against the
+oracle run on the same bf16 values in fp64; fp32 path max-abs 1e-5; span
+evaluation and ring-buffer bytes bit-exact.  Output buffers are pre-filled
+with NaN so an unwritten element fails the comparison.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from heterogeneous_sliding_window_b200 import inputs, moa
+from oracle import attention as oatt, kvcache as okv, rules as orules
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+F32_TOL = 1e-5
+DEV = "cuda"
+
+
+def _nan_like(shape, dtype):
+    return torch.full(shape, float("nan"), dtype=dtype, device=DEV)
+
+
+def _bf16_prefill(q, k, v, spans, scale, fill=None):
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    o = _nan_like((B, Hq, N, d), torch.bfloat16)
+    ws = moa.Workspace(moa.MOA_OP_PREFILL, B, Hq, N, d, spans)
+    moa.moa_prefill(q, k, v, o, B, Hq, Hkv, N, d, "bf16", spans, scale, ws.ptr, ws.nbytes,
+                    fill.handle if fill is not None else None)
+    moa.moa_workspace_check(ws.ptr)
+    torch.cuda.synchronize()
+    return o
+
+
+# ---------------------------------------------------------------------------
+# Tiny fp32 configuration: B=1, 4 heads, d=64, N=256, spans {32,64,128,256}
+# (beta = 0, block 32); full prefill, then 16 decode steps through the ring.
+# ---------------------------------------------------------------------------
+def test_tiny_fp32_prefill_fill_and_16_decode_steps():
+    B, H, d, N = 1, 4, 64, 256
+    a, b = inputs.tiny_tables()
+    spans = moa.moa_rules_eval(a, b, N, 32)
+    assert spans == orules.eval_spans(a, b, N, 32) == [32, 64, 128, 256]
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn(100, (B, H, N, d), "f32")
+    k = inputs.randn(101, (B, H, N, d), "f32")
+    v = inputs.randn(102, (B, H, N, d), "f32")
+    cache = moa.KVCache(B, H, d, "f32", spans)
+    o = _nan_like((B, H, N, d), torch.float32)
+    moa.moa_prefill(q.to(DEV), k.to(DEV), v.to(DEV), o, B, H, H, N, d, "f32", spans, scale,
+                    None, 0, cache.handle)
+    torch.cuda.synchronize()
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale)
+    assert np.max(np.abs(inputs.as_f64(o) - ref)) <= F32_TOL
+
+    ring = okv.RingCache(B, H, d, spans)
+    ring.append(inputs.as_f64(k), inputs.as_f64(v))
+    assert cache.positions() == ring.t == [N]
+    assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "f32")
+
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, spans)
+    for step in range(16):
+        qt = inputs.randn(200 + step, (B, H, d), "f32")
+        kt = inputs.randn(300 + step, (B, H, 1, d), "f32")
+        vt = inputs.randn(400 + step, (B, H, 1, d), "f32")
+        cache.append(kt.to(DEV), vt.to(DEV))
+        ot = _nan_like((B, H, d), torch.float32)
+        moa.moa_decode(cache.handle, qt.to(DEV), ot, H, spans, scale, ws.ptr, ws.nbytes)
+        torch.cuda.synchronize()
+        ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+        ref_t = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+        assert np.max(np.abs(inputs.as_f64(ot) - ref_t)) <= F32_TOL, step
+    assert cache.positions() == ring.t == [N + 16]
+    assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "f32")
+
+
+# ---------------------------------------------------------------------------
+# bf16 tensor-core prefill
+# ---------------------------------------------------------------------------
+PREFILL_CASES = [
+    # (B, Hq, Hkv, N, spans, q_gain)   -- ragged N, spans around tile edges, GQA
+    (1, 4, 4, 1000, [1, 64, 200, 1000], 1.0),
+    (2, 8, 2, 700, [1, 127, 128, 129, 256, 300, 700, 5000], 1.0),
+    (1, 2, 1, 513, [384, 100], 4.0),              # peaky scores: stresses the lazy rescale
+    (1, 3, 3, 128, [128, 1, 37], 1.0),            # exactly one tile
+    (1, 2, 2, 1, [1, 5], 1.0),                    # a single token
+    (3, 4, 4, 300, [300, 300, 300, 300], 2.0),    # dense causal (S = N)
+]
+
+
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: "B%d_H%d_%d_N%d" % c[:4])
+def test_bf16_prefill_matches_oracle(case):
+    B, Hq, Hkv, N, spans, gain = case
+    d = 128
+    scale = 1.0 / math.sqrt(d)
+    q = (inputs.randn(1, (B, Hq, N, d), "f32") * gain).to(torch.bfloat16)
+    k = inputs.randn(2, (B, Hkv, N, d))
+    v = inputs.randn(3, (B, Hkv, N, d))
+    o = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, scale)
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale)
+    err = np.max(np.abs(inputs.as_f64(o) - ref))
+    assert err <= BF16_TOL, err
+
+
+def test_bf16_prefill_fill_cache_bytes():
+    B, Hq, Hkv, N, d = 2, 4, 2, 600, 128
+    spans = [64, 256, 600, 100]
+    caps = okv.group_capacities(spans, Hkv)
+    q = inputs.randn(7, (B, Hq, N, d))
+    k = inputs.randn(8, (B, Hkv, N, d))
+    v = inputs.randn(9, (B, Hkv, N, d))
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, 0.1, fill=cache)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    ring.append(inputs.as_f64(k), inputs.as_f64(v))
+    assert cache.positions() == [N, N]
+    assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "bf16")
+
+
+def _sample_rows(B, H, N, rng, n=96):
+    rows = set()
+    for b in range(B):
+        for h in range(H):
+            for i in (0, 1, 127, 128, N - 1, N - 2):
+                if 0 <= i < N:
+                    rows.add((b, h, i))
+    rows = sorted(rows)
+    extra = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))) for _ in range(n)]
+    return rows + extra
+
+
+def test_bf16_prefill_vicuna7b_full_size_sampled():
+    """B=1, 32 heads, d=128, N=8192, 25% density spans: the bench launch, sampled rows."""
+    B, H, N, d = 1, 32, 8192, 128
+    a, b = inputs.tables_7b(1, H, N, 64, 0.25, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    assert spans == orules.eval_spans(a, b, N, 64)
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(11, (B, H, N, d))
+    k = inputs.randn_cuda(12, (B, H, N, d))
+    v = inputs.randn_cuda(13, (B, H, N, d))
+    o = _bf16_prefill(q, k, v, spans, scale)
+    assert not torch.isnan(o).any()
+    rows = _sample_rows(B, H, N, np.random.default_rng(0), n=64)
+    rows = [r for r in rows if r[1] % 4 == 0 or r[2] in (N - 1,)][:160]
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale, rows=rows)
+    got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
+    assert np.max(np.abs(got - ref)) <= BF16_TOL
+
+
+def test_bf16_prefill_llama3_gqa_dense_sampled():
+    """Hq=32 / Hkv=8, N=32768, every span = N (the dense causal check), sampled rows."""
+    B, Hq, Hkv, N, d = 1, 32, 8, 32768, 128
+    spans = [N] * Hq
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(21, (B, Hq, N, d))
+    k = inputs.randn_cuda(22, (B, Hkv, N, d))
+    v = inputs.randn_cuda(23, (B, Hkv, N, d))
+    o = _bf16_prefill(q, k, v, spans, scale)
+    rows = [(0, h, i) for h in (0, 5, 31) for i in (0, 129, 4095, 20000, N - 1)]
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale, rows=rows)
+    got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
+    assert np.max(np.abs(got - ref)) <= BF16_TOL
+
+
+# ---------------------------------------------------------------------------
+# Ring-buffer append and bf16 decode
+# ---------------------------------------------------------------------------
+def test_append_bytes_bit_exact():
+    B, Hkv, d = 3, 3, 128
+    caps = [1, 70, 300]
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    for step, n in enumerate([5, 1, 299, 1, 1, 64, 700, 1, 3]):
+        k = inputs.randn(50 + step, (B, Hkv, n, d))
+        v = inputs.randn(60 + step, (B, Hkv, n, d))
+        cache.append(k.to(DEV), v.to(DEV))
+        ring.append(inputs.as_f64(k), inputs.as_f64(v))
+        torch.cuda.synchronize()
+        assert cache.positions() == ring.t
+        assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "bf16")
+
+
+DECODE_CASES = [
+    # (B, Hq, Hkv, prefix, spans, steps)
+    (2, 4, 4, 900, [1, 256, 257, 900], 3),         # multi-split heads, single-split heads
+    (3, 8, 2, 50, [40, 7, 64, 64, 300, 1, 299, 17], 4),  # prefix shorter than spans, GQA
+    (1, 4, 1, 2000, [1000, 513, 2000, 1], 2),       # window smaller than ring: wraps
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "B%d_H%d_%d_T%d" % c[:4])
+def test_bf16_decode_matches_oracle(case):
+    B, Hq, Hkv, prefix, spans, steps = case
+    d = 128
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    k0 = inputs.randn(70, (B, Hkv, prefix, d))
+    v0 = inputs.randn(71, (B, Hkv, prefix, d))
+    cache.append(k0.to(DEV), v0.to(DEV))
+    ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    for step in range(steps):
+        qt = (inputs.randn(80 + step, (B, Hq, d), "f32") * (1 + step)).to(torch.bfloat16)
+        kt = inputs.randn(90 + step, (B, Hkv, 1, d))
+        vt = inputs.randn(95 + step, (B, Hkv, 1, d))
+        cache.append(kt.to(DEV), vt.to(DEV))
+        ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+        ot = _nan_like((B, Hq, d), torch.bfloat16)
+        moa.moa_decode(cache.handle, qt.to(DEV), ot, Hq, spans, scale, ws.ptr, ws.nbytes)
+        torch.cuda.synchronize()
+        ref = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+        err = np.max(np.abs(inputs.as_f64(ot) - ref))
+        assert err <= BF16_TOL, (step, err)
+    assert cache.positions() == ring.t
+
+
+def test_bf16_decode_vicuna7b_layer_full_size_sampled():
+    """One layer of the decode workload: B=32, 32 heads, context 4096, 50% density."""
+    B, H, d, N = 32, 32, 128, 4096
+    a, b = inputs.tables_7b(1000, H, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    cache = moa.KVCache(B, H, d, "bf16", spans)
+    data = cache.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(5, (data.numel(),)))
+    cache.set_positions([N] * B)
+    rng = np.random.default_rng(3)
+    picks = [(int(rng.integers(B)), int(rng.integers(H))) for _ in range(24)] + [(0, 0), (B - 1, H - 1)]
+    blocks = {}
+    host = None
+    for bb, hh in picks:
+        if (bb, hh) not in blocks:
+            if host is None:
+                host = cache.data_bytes().cpu().numpy().tobytes()
+            blocks[(bb, hh)] = okv.block_from_image(host, bb, hh, B, H, d, spans, "bf16")
+    scale = 1.0 / math.sqrt(d)
+    qt = inputs.randn_cuda(6, (B, H, d))
+    kt = inputs.randn_cuda(7, (B, H, 1, d))
+    vt = inputs.randn_cuda(8, (B, H, 1, d))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, spans)
+    cache.append(kt, vt)
+    ot = _nan_like((B, H, d), torch.bfloat16)
+    moa.moa_decode(cache.handle, qt, ot, H, spans, scale, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    assert cache.positions() == [N + 1] * B
+    kt64, vt64, qt64, ot64 = (inputs.as_f64(x) for x in (kt, vt, qt, ot))
+    for bb, hh in picks:
+        K, V = blocks[(bb, hh)]
+        C = spans[hh]
+        K[N % C] = kt64[bb, hh, 0]          # the appended token's slot
+        V[N % C] = vt64[bb, hh, 0]
+        ref = okv.decode_row_from_ring(K, V, N + 1, spans[hh], qt64[bb, hh], scale)
+        assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
+
+
+def test_decode_empty_sequence_sets_error_bit():
+    B, H, d = 2, 2, 128
+    cache = moa.KVCache(B, H, d, "bf16", [8, 8])
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, [8, 8])
+    q = inputs.randn_cuda(1, (B, H, d))
+    o = _nan_like((B, H, d), torch.bfloat16)
+    moa.moa_decode(cache.handle, q, o, H, [8, 8], 0.1, ws.ptr, ws.nbytes)
+    with pytest.raises(moa.MoaError) as e:
+        cache.positions()
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    assert torch.all(o.float() == 0)
+
+
+def test_decode_rejects_span_above_capacity():
+    cache = moa.KVCache(1, 1, 128, "bf16", [64])
+    ws = moa.Workspace(moa.MOA_OP_DECODE, 1, 1, 0, 128, [64])
+    q = inputs.randn_cuda(1, (1, 1, 128))
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_decode(cache.handle, q, q.clone(), 1, [65], 0.1, ws.ptr, ws.nbytes)
+    assert e.value.status == moa.MOA_ERR_CAPACITY
