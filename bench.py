@@ -278,7 +278,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     moa.moa_workspace_check(p_ws.ptr)
 
-    clocks = Clocks(torch.cuda.current_device())
+    try:
+        clocks = Clocks("GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid))
+    except Exception:
+        clocks = Clocks(torch.cuda.current_device())
     evs = [new_events() for _ in range(args.steps)]
     if dist:
         dist.barrier()
@@ -397,13 +400,28 @@ def run_ours(args):
 
 
 def _ncu_traffic():
-    """Per-launch DRAM bytes from the committed ncu summaries, if they match the current kernels."""
+    """Per-launch DRAM bytes (read + write) from the committed ncu capture of each kernel.
+
+    A kernel whose source changed since its capture (sha256 prefix mismatch) reports null.
+    """
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
+    srcs = {"decode": "decode.cu", "prefill": "prefill_sm100.cu"}
+    out = {}
     try:
         with open(path) as f:
-            return json.load(f)
+            tr = json.load(f)
     except Exception:
-        return {}
+        return out
+    for key, fname in srcs.items():
+        try:
+            with open(os.path.join(ROOT, "heterogeneous_sliding_window_b200", "csrc", fname), "rb") as f:
+                h = hashlib.sha256(f.read()).hexdigest()[:16]
+        except OSError:
+            continue
+        if tr.get("source_sha256_prefix", {}).get(key) == h:
+            out[key] = tr.get(key)
+    return out
 
 
 def run_reference(args):
@@ -429,14 +447,60 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_profile_case(case, launches=3):
+    """Small single-kernel cases for ncu captures (a few GB on the device at most).
+
+    prefill: the 7B prompt (B=1, 32 heads, N=8192; Q/K/V 192 MiB), `launches` prefills.
+    decode : one decode layer of the 7B workload (B=32, 32 heads, context 4096; 1 GiB cache).
+    """
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    moa.load()
+    if case == "prefill":
+        pa, pb = inputs.tables_7b(P_SEED, P_H, P_N, BLOCK, P_DENSITY, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(pa, pb, P_N, BLOCK)
+        q = inputs.randn_cuda(10, (P_B, P_H, P_N, P_D))
+        k = inputs.randn_cuda(11, (P_B, P_H, P_N, P_D))
+        v = inputs.randn_cuda(12, (P_B, P_H, P_N, P_D))
+        o = torch.empty_like(q)
+        ws = moa.Workspace(moa.MOA_OP_PREFILL, P_B, P_H, P_N, P_D, sp)
+        for _ in range(launches):
+            moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", sp, 1.0 / math.sqrt(P_D), ws.ptr,
+                            ws.nbytes)
+        moa.moa_workspace_check(ws.ptr)
+    else:
+        a, b = inputs.tables_7b(D_SEED, D_H, D_N, BLOCK, D_DENSITY, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, D_N, BLOCK)
+        c = moa.KVCache(D_B, D_H, D_D, "bf16", sp)
+        data = c.data_bytes().view(torch.bfloat16)
+        data.copy_(inputs.randn_cuda(100, (data.numel(),)))
+        c.set_positions([D_N] * D_B)
+        ws = moa.Workspace(moa.MOA_OP_DECODE, D_B, D_H, 0, D_D, sp)
+        q = inputs.randn_cuda(200, (D_B, D_H, D_D))
+        k = inputs.randn_cuda(300, (D_B, D_H, 1, D_D))
+        v = inputs.randn_cuda(400, (D_B, D_H, 1, D_D))
+        o = torch.empty_like(q)
+        for _ in range(launches):
+            moa.moa_kv_append(c.handle, k, v, 1)
+            moa.moa_decode(c.handle, q, o, D_H, sp, 1.0 / math.sqrt(D_D), ws.ptr, ws.nbytes)
+        c.positions()
+    torch.cuda.synchronize()
+    print("profile case %s done" % case)
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+                    help="run one small single-kernel case (for ncu) and exit")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         args.warmup = 3
     res = run_reference(args) if args.impl == "reference" else run_ours(args)
