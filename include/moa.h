@@ -189,6 +189,32 @@ moa_status moa_decode(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
                       const int32_t* spans, float scale, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Decode without a caller workspace.  The paper has no counterpart: this is
+ * a deployment convenience of this library.
+ *
+ * Same computation, arguments and errors as moa_decode, minus the workspace.
+ * It is for callers that cannot allocate device memory -- e.g. an operator
+ * plugin that its host framework gives only input and output pointers, a
+ * runtime whose device memory is entirely owned by another allocator, or code
+ * that must not call cudaMalloc because that call synchronises the device.
+ * The split partials and tickets live instead in one fixed 8 MiB scratch
+ * array inside libmoa's device image, which every GPU that loads the library
+ * keeps until the process exits.  The caller still passes q, o and the cache.
+ *  - Requests whose decode workspace (moa_workspace_bytes(MOA_OP_DECODE, ...))
+ *    exceeds 8 MiB return MOA_ERR_WORKSPACE and launch nothing.
+ *  - The first call on each device looks up the array's device address with
+ *    that device current (cudaGetSymbolAddress); make that first call before
+ *    any stream capture.
+ *  - Each call clears the array's tickets on `stream`, then launches the
+ *    decode kernel; the array keeps the last call's partials.  All calls on a
+ *    device share the array, so calls whose work overlaps on the GPU (other
+ *    streams, unordered threads) race and may return wrong outputs.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * ------------------------------------------------------------------------- */
+moa_status moa_decode_static_ws(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
+                                const int32_t* spans, float scale, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
