@@ -1,6 +1,8 @@
 // C ABI front end of libmoa: argument validation and dispatch to the kernels.
 // Every check that can fail does so here, on the host, before anything is
 // enqueued; the kernels assume validated arguments.
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 
@@ -14,6 +16,12 @@ int sm_count() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return 148;
   return n;
+}
+
+moa_status cuda_fail(cudaError_t e, const char* where) {
+  static const bool verbose = std::getenv("MOA_VERBOSE") != nullptr;
+  if (verbose) std::fprintf(stderr, "libmoa: %s: %s\n", where, cudaGetErrorString(e));
+  return MOA_ERR_CUDA;
 }
 
 }  // namespace moa
@@ -165,22 +173,34 @@ extern "C" moa_status moa_workspace_check(const void* ws, void* stream) {
 }
 
 extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
-                                           int32_t* units_out, int64_t cap, int64_t* n_units_out) {
-  if (B < 1 || Hq < 1 || Hq > MOA_MAX_HEADS || N < 1 || N > INT32_MAX || !spans || !n_units_out ||
-      cap < 0 || (cap > 0 && !units_out))
+                                           int32_t* rows_out, int64_t cap, int64_t* n_rows_out) {
+  if (B < 1 || Hq < 1 || Hq > MOA_MAX_HEADS || N < 1 || N > INT32_MAX || !spans || !n_rows_out ||
+      cap < 0 || (cap > 0 && !rows_out))
     return MOA_ERR_INVALID_ARG;
   for (int32_t h = 0; h < Hq; ++h)
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
   std::vector<int32_t> u = prefill_units(B, Hq, (int32_t)N, spans);
-  const int64_t n = (int64_t)u.size() / 4;
-  *n_units_out = n;
-  for (int64_t i = 0; i < n && i < cap; ++i) {
-    units_out[5 * i + 0] = u[4 * i + 0];
-    units_out[5 * i + 1] = u[4 * i + 1];
-    units_out[5 * i + 2] = u[4 * i + 2];
-    units_out[5 * i + 3] = u[4 * i + 3];
-    units_out[5 * i + 4] = u[4 * i + 2];  // hi: the diagonal tile
+  const int64_t n_units = (int64_t)u.size() / 4;
+  int64_t n = 0;
+  for (int64_t i = 0; i < n_units; ++i) {
+    int32_t t[4];
+    const int32_t b = u[4 * i], h = u[4 * i + 1], mp = u[4 * i + 2];
+    prefill_unit_tiles((int32_t)N, spans[h], mp, t);
+    for (int x = 0; x < 2; ++x) {
+      if (t[2 * x + 1] < 0) continue;
+      if (n < cap) {
+        int32_t* r = rows_out + 6 * n;
+        r[0] = (int32_t)i;
+        r[1] = b;
+        r[2] = h;
+        r[3] = t[2 * x + 1];   // query tile m
+        r[4] = t[2 * x];       // lo
+        r[5] = t[2 * x + 1];   // hi: the diagonal tile
+      }
+      ++n;
+    }
   }
+  *n_rows_out = n;
   return MOA_OK;
 }
 

@@ -315,7 +315,7 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
     if (c->d == 128) decode_kernel<float, 128><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
     else decode_kernel<float, 64><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
   }
-  return cudaGetLastError() == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
+  return check_launch("decode launch");
 }
 
 }  // namespace moa

@@ -38,6 +38,14 @@ constexpr uint32_t kErrEmpty = 2u;
 
 int sm_count();
 
+// MOA_ERR_CUDA with the CUDA error reported on stderr when the environment
+// variable MOA_VERBOSE is set (the status alone cannot carry the reason).
+moa_status cuda_fail(cudaError_t e, const char* where);
+inline moa_status check_launch(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOA_OK : cuda_fail(e, where);
+}
+
 // kv.cu
 moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
                          cudaStream_t s);
@@ -56,8 +64,10 @@ moa_status launch_prefill_f32(const float* q, const float* k, const float* v, fl
 // prefill_sm100.cu (bf16, tcgen05)
 constexpr int kTileM = 128;   // query rows per work unit
 constexpr int kTileN = 128;   // keys per key/value tile
-struct Unit { int32_t b, h, m, lo; };     // key tiles lo..m (the diagonal tile is m)
 std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans);
+// Key-tile ranges of unit mp's two query tiles: {loA, hiA, loB, hiB}; B = -1 when
+// its query tile lies beyond N.
+void prefill_unit_tiles(int32_t N, int32_t S, int32_t mp, int32_t tiles[4]);
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,
                                int32_t B, int32_t Hq, int32_t Hkv, int32_t N,

@@ -90,7 +90,7 @@ moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t 
   }
   dim3 grid((maxrows + kAppendRows - 1) / kAppendRows, c->Hkv, c->B);
   append_kernel<<<grid, kAppendThreads, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
+  return check_launch("append launch");
 }
 
 }  // namespace moa

@@ -85,7 +85,7 @@ moa_status launch_prefill_f32(const float* q, const float* k, const float* v, fl
   dim3 grid((N + kRowsPerBlock - 1) / kRowsPerBlock, Hq, B);
   if (d == 128) prefill_f32_kernel<128><<<grid, 32 * kRowsPerBlock, 0, s>>>(p);
   else prefill_f32_kernel<64><<<grid, 32 * kRowsPerBlock, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
+  return check_launch("prefill_f32 launch");
 }
 
 }  // namespace moa

@@ -208,7 +208,7 @@ def moa_prefill_schedule(B, Hq, N, spans):
     sp, spp = _i32(spans)
     n = ctypes.c_int64()
     _check(load().moa_prefill_schedule(B, Hq, int(N), spp, None, 0, ctypes.byref(n)), "moa_prefill_schedule")
-    out = np.zeros((n.value, 5), dtype=np.int32)
+    out = np.zeros((n.value, 6), dtype=np.int32)
     _check(load().moa_prefill_schedule(B, Hq, int(N), spp, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                                        n.value, ctypes.byref(n)), "moa_prefill_schedule")
     return out

@@ -92,23 +92,28 @@ def _tiles_needed_brute(m, S, N):
 
 
 @pytest.mark.parametrize("N,spans", [(1000, [1, 64, 127, 128, 129, 300, 1000, 5000]), (128, [1, 128]),
-                                     (129, [2, 129]), (5, [3])])
+                                     (129, [2, 129]), (5, [3]), (640, [256, 700])])
 def test_prefill_schedule_covers_band(N, spans):
     B = 2
     Hq = len(spans)
-    units = moa.moa_prefill_schedule(B, Hq, N, spans)
+    rows = moa.moa_prefill_schedule(B, Hq, N, spans)
     M = (N + 127) // 128
-    assert units.shape == (B * Hq * M, 5)
+    assert rows.shape == (B * Hq * M, 6)
     seen = set()
-    costs = []
-    for b, h, m, lo, hi in units.tolist():
+    unit_cost = {}
+    order = []
+    for unit, b, h, m, lo, hi in rows.tolist():
         assert (b, h, m) not in seen
         seen.add((b, h, m))
         assert hi == m
         need = _tiles_needed_brute(m, spans[h], N)
         assert set(range(lo, hi + 1)) == need   # exactly the band's tiles, none skipped, none extra
-        costs.append(hi - lo + 1)
+        unit_cost[unit] = unit_cost.get(unit, 0) + hi - lo + 1
+        if not order or order[-1] != unit:
+            order.append(unit)
     assert len(seen) == B * Hq * M
+    assert order == sorted(order)               # rows of a unit are adjacent
+    costs = [unit_cost[u] for u in order]
     assert costs == sorted(costs, reverse=True)  # longest first
 
 
@@ -158,7 +163,7 @@ def test_workspace_sizes():
     d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)
     p = moa.moa_workspace_bytes(moa.MOA_OP_PREFILL, 2, 4, 1000, 128, spans)
     assert d % 256 == 0 and d >= 256 + 2 * 4 * 4
-    assert p >= 256 + 2 * 4 * 8 * 16
+    assert p >= 256 + 2 * 4 * 4 * 16   # units of two 128-row query tiles
     with pytest.raises(moa.MoaError):
         moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, [64, 0, 1, 1])
 
