@@ -65,9 +65,10 @@ constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizz
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
 constexpr uint32_t OFF_QA = 0;
 constexpr uint32_t OFF_QB = OFF_QA + kTileBytes;
-constexpr uint32_t OFF_K = OFF_QB + kTileBytes;       // 2 stages
-constexpr uint32_t OFF_V = OFF_K + 2 * kTileBytes;    // 2 stages
-constexpr uint32_t OFF_BAR = OFF_V + 2 * kTileBytes;
+constexpr uint32_t kKStages = 2, kVStages = 2;        // K and V ring depths
+constexpr uint32_t OFF_K = OFF_QB + kTileBytes;
+constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
+constexpr uint32_t OFF_BAR = OFF_V + kVStages * kTileBytes;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024; // + barriers + alignment slack
 
 constexpr uint32_t kTmemCols = 512;   // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
@@ -79,14 +80,25 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 
 // mbarrier slots (8 bytes each) at OFF_BAR
 enum {
-  B_QFULL = 0, B_QEMPTY, B_KFULL0, B_KFULL1, B_KEMPTY0, B_KEMPTY1, B_VFULL0, B_VFULL1,
-  B_VEMPTY0, B_VEMPTY1, B_SFULL_A, B_SFULL_B, B_PFULL_A, B_PFULL_B, B_OFULL_A, B_OFULL_B,
-  B_OEMPTY_A, B_OEMPTY_B, B_UFULL0, B_UFULL1, B_UEMPTY0, B_UEMPTY1, B_COUNT
+  B_QFULL = 0, B_QEMPTY, B_SFULL_A, B_SFULL_B, B_PFULL_A, B_PFULL_B, B_OFULL_A, B_OFULL_B,
+  B_OEMPTY_A, B_OEMPTY_B, B_UFULL0, B_UFULL1, B_UEMPTY0, B_UEMPTY1,
+  B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
+  B_COUNT = B_VEMPTY0 + 4
+};
+static_assert(kKStages <= 4 && kVStages <= 4, "ring depth");
+
+// Position in a ring of `n` stages: stage index and mbarrier phase parity.
+struct Ring {
+  uint32_t stage = 0, phase = 0;
+  __device__ void next(uint32_t n) {
+    if (++stage == n) { stage = 0; phase ^= 1u; }
+  }
 };
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
 constexpr uint32_t OFF_UNIT = OFF_ABORT + 4;                     // int[2]
 static_assert(OFF_UNIT + 8 <= OFF_BAR + 512, "barrier area");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct PrefillParams {
   uint32_t* hdr;                 // [0] error word, [1] unit counter
@@ -191,8 +203,7 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
       float s[128];
       {
         uint32_t sr[128];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + cc * 32, sr + cc * 32);
+        tmem_ld128(tS, sr);
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc) s[cc] = __uint_as_float(sr[cc]);
       }
@@ -204,9 +215,14 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
         for (int cc = 0; cc < 128; ++cc)
           if (cc > hi_c || cc <= lo_c) s[cc] = -INFINITY;
       }
-      float tmax = fmaxf(s[0], s[1]);
+      float mx[8];                                   // 8 independent max chains
 #pragma unroll
-      for (int cc = 2; cc < 128; cc += 2) tmax = max3(tmax, s[cc], s[cc + 1]);
+      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+      for (int cc = 16; cc < 128; cc += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], s[cc + 2 * k], s[cc + 2 * k + 1]);
+      const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float mt = tmax * p.scale_log2;
       const float m_old = m_run;
       const bool rescale = mt > m_run + kRescaleThreshold;
@@ -230,21 +246,26 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
           tmem_st32(tO + cc * 32, rr);
         }
       }
-      // exponentials, row sum, P (bf16 pairs) into TMEM over S
-      float lsum = 0.f;
+      // exponentials (MUFU ex2), row sum in 8 independent chains, P (bf16
+      // pairs) into TMEM over S
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {               // 2 x 32 columns = 128 keys
         uint32_t w[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = ex2_approx(fmaf(s[cc * 64 + 2 * j], p.scale_log2, neg));
-          const float p1 = ex2_approx(fmaf(s[cc * 64 + 2 * j + 1], p.scale_log2, neg));
-          lsum += p0 + p1;
+          const float x0 = fmaf(s[cc * 64 + 2 * j], p.scale_log2, neg);
+          const float x1 = fmaf(s[cc * 64 + 2 * j + 1], p.scale_log2, neg);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          ls[j & 7] += p0 + p1;
           w[j] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tS + cc * 32, w);
       }
-      l_run += lsum;
+      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(c.bar(B_PFULL_A + X));
@@ -290,7 +311,8 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t sV, 
 
 __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
                                          uint32_t sQ0, uint32_t sK0, uint32_t sV0) {
-  uint32_t kc = 0, vc = 0, qc = 0;          // K tiles, V tiles, units consumed
+  Ring kr, vr;                              // K and V ring positions
+  uint32_t qc = 0;                          // units consumed
   uint32_t pc[2] = {0, 0}, oe[2] = {0, 0};  // P tiles consumed, units started per X
   for (uint32_t i = 0;; ++i) {
     if (!c.wait(B_UFULL0 + (i & 1), (i >> 1) & 1)) return;
@@ -306,14 +328,14 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     bool first_pv[2] = {true, true};
     uint32_t v_prev = 0;                   // V stage of key tile kt-1
     for (int kt = lo; kt <= hi; ++kt) {
-      const uint32_t ks = kc & 1;
-      if (!c.wait(B_KFULL0 + ks, (kc >> 1) & 1)) return;
-      ++kc;
+      const uint32_t ks = kr.stage;
+      if (!c.wait(B_KFULL0 + ks, kr.phase)) return;
+      kr.next(kKStages);
       tc_fence_after();
       if (kt > lo) {                       // V(kt-1) feeds this step's PVs
-        v_prev = vc & 1;
-        if (!c.wait(B_VFULL0 + v_prev, (vc >> 1) & 1)) return;
-        ++vc;
+        v_prev = vr.stage;
+        if (!c.wait(B_VFULL0 + v_prev, vr.phase)) return;
+        vr.next(kVStages);
         tc_fence_after();
       }
 #pragma unroll
@@ -348,9 +370,9 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     }
     mma_commit(c.bar(B_QEMPTY));           // every S of the unit is issued
     // tail: PVs of the last key tile
-    v_prev = vc & 1;
-    if (!c.wait(B_VFULL0 + v_prev, (vc >> 1) & 1)) return;
-    ++vc;
+    v_prev = vr.stage;
+    if (!c.wait(B_VFULL0 + v_prev, vr.phase)) return;
+    vr.next(kVStages);
     tc_fence_after();
 #pragma unroll
     for (int X = 0; X < 2; ++X) {
@@ -381,7 +403,8 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
                                               const CUtensorMap* tmQ, const CUtensorMap* tmK,
                                               const CUtensorMap* tmV, uint32_t sQ0, uint32_t sK0,
                                               uint32_t sV0) {
-  uint32_t kc = 0, vc = 0, qc = 0;
+  Ring kr, vr;
+  uint32_t qc = 0;
   for (uint32_t i = 0;; ++i) {
     if (!c.wait(B_UEMPTY0 + (i & 1), ((i >> 1) & 1) ^ 1)) return;
     const int u = (int)atomicAdd(p.hdr + 1, 1u);
@@ -401,15 +424,15 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
       tma_load_3d(sQ0 + kTileBytes + kHalfBytes, tmQ, c.bar(B_QFULL), 64, x.hiB * 128, x.zq);
     }
     for (int kt = lo; kt <= hi; ++kt) {
-      const uint32_t ks = kc & 1;
-      if (!c.wait(B_KEMPTY0 + ks, ((kc >> 1) & 1) ^ 1)) return;
-      ++kc;
+      const uint32_t ks = kr.stage;
+      if (!c.wait(B_KEMPTY0 + ks, kr.phase ^ 1)) return;
+      kr.next(kKStages);
       mbar_expect_tx(c.bar(B_KFULL0 + ks), kTileBytes);
       tma_load_3d(sK0 + ks * kTileBytes, tmK, c.bar(B_KFULL0 + ks), 0, kt * 128, x.zk);
       tma_load_3d(sK0 + ks * kTileBytes + kHalfBytes, tmK, c.bar(B_KFULL0 + ks), 64, kt * 128, x.zk);
-      const uint32_t vs = vc & 1;
-      if (!c.wait(B_VEMPTY0 + vs, ((vc >> 1) & 1) ^ 1)) return;
-      ++vc;
+      const uint32_t vs = vr.stage;
+      if (!c.wait(B_VEMPTY0 + vs, vr.phase ^ 1)) return;
+      vr.next(kVStages);
       mbar_expect_tx(c.bar(B_VFULL0 + vs), kTileBytes);
       tma_load_3d(sV0 + vs * kTileBytes, tmV, c.bar(B_VFULL0 + vs), 0, kt * 128, x.zk);
       tma_load_3d(sV0 + vs * kTileBytes + kHalfBytes, tmV, c.bar(B_VFULL0 + vs), 64, kt * 128, x.zk);
