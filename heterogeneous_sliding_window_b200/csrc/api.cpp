@@ -180,25 +180,15 @@ extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, con
   for (int32_t h = 0; h < Hq; ++h)
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
   std::vector<int32_t> u = prefill_units(B, Hq, (int32_t)N, spans);
-  const int64_t n_units = (int64_t)u.size() / 4;
-  int64_t n = 0;
-  for (int64_t i = 0; i < n_units; ++i) {
-    int32_t t[4];
-    const int32_t b = u[4 * i], h = u[4 * i + 1], mp = u[4 * i + 2];
-    prefill_unit_tiles((int32_t)N, spans[h], mp, t);
-    for (int x = 0; x < 2; ++x) {
-      if (t[2 * x + 1] < 0) continue;
-      if (n < cap) {
-        int32_t* r = rows_out + 6 * n;
-        r[0] = (int32_t)i;
-        r[1] = b;
-        r[2] = h;
-        r[3] = t[2 * x + 1];   // query tile m
-        r[4] = t[2 * x];       // lo
-        r[5] = t[2 * x + 1];   // hi: the diagonal tile
-      }
-      ++n;
-    }
+  const int64_t n = (int64_t)u.size() / 4;
+  for (int64_t i = 0; i < n && i < cap; ++i) {
+    int32_t* r = rows_out + 6 * i;
+    r[0] = (int32_t)i;
+    r[1] = u[4 * i];
+    r[2] = u[4 * i + 1];
+    r[3] = u[4 * i + 2];   // query tile m
+    r[4] = u[4 * i + 3];   // lo
+    r[5] = u[4 * i + 2];   // hi: the diagonal tile
   }
   *n_rows_out = n;
   return MOA_OK;

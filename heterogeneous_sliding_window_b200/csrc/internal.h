@@ -65,9 +65,7 @@ moa_status launch_prefill_f32(const float* q, const float* k, const float* v, fl
 constexpr int kTileM = 128;   // query rows per work unit
 constexpr int kTileN = 128;   // keys per key/value tile
 std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans);
-// Key-tile ranges of unit mp's two query tiles: {loA, hiA, loB, hiB}; B = -1 when
-// its query tile lies beyond N.
-void prefill_unit_tiles(int32_t N, int32_t S, int32_t mp, int32_t tiles[4]);
+
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,
                                int32_t B, int32_t Hq, int32_t Hkv, int32_t N,

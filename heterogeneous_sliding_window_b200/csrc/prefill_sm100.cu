@@ -6,34 +6,34 @@
 // applied to v_j.  Heads differ only in S_h.
 //
 // How (B200 design, not the pages' A100 kernel):
-//  * Work unit = (b, h, mp): two query tiles A = rows [256mp, 256mp+128) and
-//    B = rows [256mp+128, 256mp+256) of one head.  Because the window is a
-//    band, tile X needs exactly the key tiles loX..hiX (hiX its diagonal tile,
-//    loX = floor(max(0, 128*tileX - S_h + 1) / 128)); every other key tile is
-//    skipped.  The two query tiles share every K/V tile they both need.
+//  * Work unit = (b, h, m): query rows [128m, 128m+128) of one head.  Because
+//    the window is a band, the unit needs exactly the key tiles lo..m
+//    (lo = floor(max(0, 128m - S_h + 1) / 128)); every other key tile is
+//    skipped.
 //  * Units are sorted longest-first on the host and handed out by a
 //    persistent grid (one CTA per SM): a producer thread takes the next unit
 //    from an atomic counter and publishes it through a two-slot ring in
 //    shared memory, so heads with very different spans balance across SMs.
-//  * Warp roles (384 threads; warps 2-3 idle):
-//      warp 0      TMA producer: Q_A, Q_B once per unit; K and V tiles through
-//                  two-stage rings (128-byte swizzle).
-//      warp 1      MMA issuer (one thread): S_X = Q_X K^T and O_X += P_X V with
-//                  tcgen05.mma (M=128, N=128, K=16 steps), fp32 accumulators
-//                  in tensor memory: S_A, S_B, O_A, O_B = 4 x 128 columns.
-//      warps 4-7   softmax for tile A, warps 8-11 for tile B: one thread per
-//                  query row reads its S row from TMEM, masks only tiles that
-//                  cross the diagonal or the window's lower edge, runs the
-//                  online softmax in the exp2 domain with a lazy rescale (the
-//                  running max used for the exponentials moves only when it
-//                  would grow by more than 2^8), and writes P as bf16 back into
-//                  tensor memory over S; the PV MMA reads P from there (A
-//                  operand in TMEM) and V straight from its TMA tile (MN-major).
-//    The MMA thread alternates A and B, so the tensor core works on one query
-//    tile while the other tile's exponentials run.
-//  * Epilogue: each softmax thread normalises its O row (fp32 -> bf16,
-//    round to nearest even) and stores it; rows >= N are dropped, and
-//    out-of-range TMA rows read as zeros.
+//  * Warp roles (384 threads, setmaxnreg split 144 / 216 / 144):
+//      warp 0       TMA producer: Q once per unit into one of two buffers
+//                   (the next unit's Q loads while this unit runs), K and V
+//                   tiles through two-stage rings (128-byte swizzle).
+//      warp 1       MMA issuer (one thread), tcgen05.mma M=128, N=128, K=16:
+//                   S(k) = Q K(k)^T into one of two S buffers in tensor memory,
+//                   O += P(k-1) V(k-1) with P read from tensor memory.  S(k+1)
+//                   is issued right after PV(k-1), without waiting for the
+//                   softmax of tile k, so the tensor core works on the next
+//                   tile while the current tile's exponentials run.
+//      warps 4-7    softmax: one thread per query row reads its S row, masks
+//                   only tiles that cross the diagonal or the window's lower
+//                   edge, takes exponentials against the row's running maximum
+//                   (exact tile maxima only when needed, see softmax_role),
+//                   and writes P as bf16 pairs back over its S buffer.
+//      warps 8-11   epilogue: O / l -> bf16 (round to nearest even) -> global,
+//                   from one of two O buffers, so the next unit's PVs proceed
+//                   while the previous unit is written out.
+//    Tensor memory: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+//  * Rows >= N are dropped at the store; out-of-range TMA rows read as zeros.
 //  * Every mbarrier wait is bounded (2 s of globaltimer, or earlier if another
 //    role gave up); on a timeout the kernel sets the workspace error word,
 //    lets every role leave, waits for its in-flight copies, frees TMEM and
@@ -55,37 +55,44 @@ using namespace sm100;
 
 constexpr int kThreads = 384;                    // 3 warpgroups
 // Register split (setmaxnreg): the block launches with 384 x 168 registers;
-// warpgroup 0 (producer, MMA issuer, two idle warps) drops to 104 and the two
-// softmax warpgroups rise to 200: 128*104 + 256*200 = 64512 = 384*168.
-constexpr uint32_t kRegsLaunch = 168, kRegsControl = 104, kRegsSoftmax = 200;
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+// warpgroup 0 (producer, MMA issuer, two idle warps) and the epilogue
+// warpgroup drop to 144, the softmax warpgroup rises to 216.
+constexpr uint32_t kRegsLaunch = 168, kRegsControl = 144, kRegsSoftmax = 216, kRegsEpilogue = 144;
+static_assert(128 * (kRegsControl + kRegsSoftmax + kRegsEpilogue) <= kThreads * kRegsLaunch,
+              "register split");
 constexpr int kD = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one 128 x 128 bf16 tile
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizzled half
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
-constexpr uint32_t OFF_QA = 0;
-constexpr uint32_t OFF_QB = OFF_QA + kTileBytes;
 constexpr uint32_t kKStages = 2, kVStages = 2;        // K and V ring depths
-constexpr uint32_t OFF_K = OFF_QB + kTileBytes;
+constexpr uint32_t OFF_Q = 0;                         // two Q buffers (units alternate)
+constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;
 constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
-constexpr uint32_t OFF_BAR = OFF_V + kVStages * kTileBytes;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024; // + barriers + alignment slack
+constexpr uint32_t OFF_INVL = OFF_V + kVStages * kTileBytes;   // float[2][128]
+constexpr uint32_t OFF_BAR = OFF_INVL + 2 * 128 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;          // + barriers + alignment slack
 
-constexpr uint32_t kTmemCols = 512;   // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;        // 2 s per wait
-constexpr float kRescaleThreshold = 8.0f;             // log2 of the largest tolerated growth
 
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 
 // mbarrier slots (8 bytes each) at OFF_BAR
 enum {
-  B_QFULL = 0, B_QEMPTY, B_SFULL_A, B_SFULL_B, B_PFULL_A, B_PFULL_B, B_OFULL_A, B_OFULL_B,
-  B_OEMPTY_A, B_OEMPTY_B, B_UFULL0, B_UFULL1, B_UEMPTY0, B_UEMPTY1,
+  B_QFULL0 = 0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_PVDONE,
+  B_OFULL0, B_OFULL1,
+  B_LFULL0, B_LFULL1, B_OEMPTY0, B_OEMPTY1, B_UFULL0, B_UFULL1, B_UEMPTY0, B_UEMPTY1,
   B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
   B_COUNT = B_VEMPTY0 + 4
 };
 static_assert(kKStages <= 4 && kVStages <= 4, "ring depth");
+constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
+constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
+constexpr uint32_t OFF_UNIT = OFF_ABORT + 4;                     // int[2]
+static_assert(OFF_UNIT + 8 <= OFF_BAR + 512, "barrier area");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // Position in a ring of `n` stages: stage index and mbarrier phase parity.
 struct Ring {
@@ -94,17 +101,12 @@ struct Ring {
     if (++stage == n) { stage = 0; phase ^= 1u; }
   }
 };
-constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
-constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
-constexpr uint32_t OFF_UNIT = OFF_ABORT + 4;                     // int[2]
-static_assert(OFF_UNIT + 8 <= OFF_BAR + 512, "barrier area");
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct PrefillParams {
   uint32_t* hdr;                 // [0] error word, [1] unit counter
-  const int4* units;             // (b, h, mp, unused), longest first
+  const int4* units;             // (b, h, m, lo), longest first
   void* o;
-  int32_t n_units, N, Hq, Hkv, G, n_qtiles;
+  int32_t n_units, N, Hq, Hkv, G;
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
 };
@@ -142,64 +144,124 @@ struct Ctx {
       }
     }
   }
+  // Warp-wide roles: every lane waits, then the warp agrees on the outcome
+  // (all lanes are present), so no lane leaves while the others go on to a
+  // warp-collective tcgen05 instruction.
+  __device__ bool wait_warp(int i, uint32_t parity) const {
+    const bool ok = wait(i, parity);
+    return !__any_sync(0xffffffffu, !ok);
+  }
+  // Next unit index from the ring.  Single-thread roles (warp_wide = false)
+  // release the slot themselves; warp-wide roles release it from lane 0 after
+  // every lane has read it.
+  __device__ bool next_unit(uint32_t i, int lane, bool warp_wide, int* u) const {
+    if (warp_wide) {
+      if (!wait_warp(B_UFULL0 + (i & 1), (i >> 1) & 1)) return false;
+      *u = ring[i & 1];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_UEMPTY0 + (i & 1)));
+    } else {
+      if (!wait(B_UFULL0 + (i & 1), (i >> 1) & 1)) return false;
+      *u = ring[i & 1];
+      mbar_arrive(bar(B_UEMPTY0 + (i & 1)));
+    }
+    return true;
+  }
 };
 
-// First key tile needed by query tile `qt` under span S.
-__device__ __forceinline__ int first_key_tile(int qt, int S) {
-  const int first_key = max(0, qt * 128 - S + 1);
-  return first_key >> 7;
-}
-
 struct UnitInfo {
-  int S, zq, zk;
-  int loA, hiA, loB, hiB;
-  bool actB;
+  int S, zq, zk, m, lo;
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, int u) {
   UnitInfo x;
   const int4 U = p.units[u];
-  const int b = U.x, h = U.y, mp = U.z;
-  x.S = p.span[h];
-  x.zq = b * p.Hq + h;
-  x.zk = b * p.Hkv + h / p.G;
-  x.hiA = 2 * mp;
-  x.loA = first_key_tile(x.hiA, x.S);
-  x.hiB = x.hiA + 1;
-  x.loB = first_key_tile(x.hiB, x.S);
-  x.actB = x.hiB < p.n_qtiles;
+  x.S = p.span[U.y];
+  x.zq = U.x * p.Hq + U.y;
+  x.zk = U.x * p.Hkv + U.y / p.G;
+  x.m = U.z;
+  x.lo = U.w;
   return x;
 }
 
 // ---------------------------------------------------------------------------
-// Softmax role: 128 threads own the 128 rows of query tile X.
+// Softmax role: 128 threads own the 128 rows of the unit's query tile.
+//
+// Exponentials are taken against the running maximum m of the row (log2
+// domain) without first reducing the tile: a tile whose largest score exceeds
+// m by more than 15 makes the tile's sum of 2^(s - m) reach 2^15, and only
+// then (rarely after the first tile) is the tile's exact maximum computed, m
+// raised, the row sum and O rescaled, and the tile redone.  Every exponential
+// is therefore at most 2^15, far inside fp32 and bf16 range, and O / l is
+// exact whichever m was used.  A row with no maximum yet (first tile with
+// in-window keys) takes the exact maximum directly.
 // ---------------------------------------------------------------------------
+constexpr float kTileSumLimit = 32768.f;             // 2^15
+
+// Row maximum of 128 scores, 8 independent chains.
+__device__ __forceinline__ float row_max128(const float* s) {
+  float mx[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+  for (int cc = 16; cc < 128; cc += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], s[cc + 2 * k], s[cc + 2 * k + 1]);
+  return max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
+// p = 2^(s * c - m) for 128 scores as bf16 pairs w[64] (MUFU ex2); returns
+// the fp32 sum.
+__device__ __forceinline__ float exp_tile(const float* s, float c, float neg, uint32_t* w) {
+  const uint64_t c2 = f2_pack(c, c), n2 = f2_pack(neg, neg);
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int j = 0; j < 64; ++j) {
+    const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, n2);
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    acc[j & 3] = f2_add(acc[j & 3], p2);
+    float p0, p1;
+    f2_unpack(p2, p0, p1);
+    w[j] = pack_bf16x2(p0, p1);
+  }
+  const uint64_t t = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+  float a, b;
+  f2_unpack(t, a, b);
+  return a + b;
+}
+
+__device__ __forceinline__ void mask_tile(float* s, int hi_c, int lo_c) {
+  if (hi_c < 127 || lo_c >= 0) {
+#pragma unroll
+    for (int cc = 0; cc < 128; ++cc)
+      if (cc > hi_c || cc <= lo_c) s[cc] = -INFINITY;
+  }
+}
+
 __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
-                                             int X, int warp, int lane) {
+                                             float* inv_l, int warp, int lane) {
   const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
   const int r = quarter * 32 + lane;                 // row within the query tile
   const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-  const uint32_t tS = tmem + lane_base + (uint32_t)(X * 128);
-  const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(X * 128);
-  uint32_t s_cnt = 0, o_cnt = 0;
+  const float sc = p.scale_log2;
+  uint32_t tcount = 0, uc = 0;
   for (uint32_t i = 0;; ++i) {
-    if (!c.wait(B_UFULL0 + (i & 1), (i >> 1) & 1)) return;
-    const int u = c.ring[i & 1];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(c.bar(B_UEMPTY0 + (i & 1)));
+    int u;
+    if (!c.next_unit(i, lane, true, &u)) return;
     if (u >= p.n_units) return;
     const UnitInfo x = decode_unit(p, u);
-    if (X == 1 && !x.actB) continue;
-    const int qt = X == 0 ? x.hiA : x.hiB;
-    const int lo = X == 0 ? x.loA : x.loB;
-    const int i_row = qt * 128 + r;
-
+    const uint32_t tO = tmem + lane_base + kColO + 128u * (uc & 1);
+    const int i_row = x.m * 128 + r;
     float m_run = -INFINITY, l_run = 0.f;
-    for (int kt = lo; kt <= qt; ++kt) {
-      if (!c.wait(B_SFULL_A + X, s_cnt & 1)) return;
-      ++s_cnt;
+    for (int kt = x.lo; kt <= x.m; ++kt, ++tcount) {
+      const uint32_t sb = tcount & 1;
+      const uint32_t tS = tmem + lane_base + kColS + 128u * sb;
+      if (!c.wait_warp(B_SFULL0 + sb, (tcount >> 1) & 1)) return;
       tc_fence_after();
-      __syncwarp();
+      const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
+      const int lo_c = i_row - x.S - kt * 128;       // keys c >  lo_c are inside the window
       float s[128];
       {
         uint32_t sr[128];
@@ -207,76 +269,79 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc) s[cc] = __uint_as_float(sr[cc]);
       }
-      // mask: only tiles crossing the diagonal or the window's lower edge
-      const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
-      const int lo_c = i_row - x.S - kt * 128;       // keys c >  lo_c are inside the window
-      if (hi_c < 127 || lo_c >= 0) {
-#pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
-          if (cc > hi_c || cc <= lo_c) s[cc] = -INFINITY;
+      mask_tile(s, hi_c, lo_c);
+      // rows without a maximum yet take this tile's exact maximum
+      const bool need_max = m_run == -INFINITY;
+      if (__any_sync(0xffffffffu, need_max)) {
+        const float tmax = row_max128(s);
+        if (need_max) m_run = tmax * sc;            // stays -inf if every key is masked
       }
-      float mx[8];                                   // 8 independent max chains
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[2 * k], s[2 * k + 1]);
-#pragma unroll
-      for (int cc = 16; cc < 128; cc += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], s[cc + 2 * k], s[cc + 2 * k + 1]);
-      const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float mt = tmax * p.scale_log2;
-      const float m_old = m_run;
-      const bool rescale = mt > m_run + kRescaleThreshold;
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx(m_old - mt);              // 0 when m_old = -inf
-        m_run = mt;
-        l_run *= alpha;
-      }
-      const float neg = (m_run == -INFINITY) ? 0.f : -m_run;
-      // O_X is stable here: PV_X(kt-1) completed before S_X(kt) (in-order MMAs).
-      const bool o_rescale = rescale && (m_old != -INFINITY) && kt > lo;
-      if (__any_sync(0xffffffffu, o_rescale)) {
-        const float a = o_rescale ? alpha : 1.f;
+      uint32_t w[64];
+      float l_tile = exp_tile(s, sc, m_run == -INFINITY ? 0.f : -m_run, w);
+      const bool redo = !(l_tile < kTileSumLimit);
+      if (__any_sync(0xffffffffu, redo)) {
+        // Rare: a score far above the running maximum.  Take the tile's exact
+        // maximum, rescale the row, and recompute the tile.
+        const float mt = row_max128(s) * sc;
+        float alpha = 1.f;
+        if (redo) {
+          alpha = ex2_approx(m_run - mt);
+          m_run = mt;
+          l_run *= alpha;
+        }
+        if (__any_sync(0xffffffffu, redo && kt > x.lo)) {
+          // O must hold every PV up to tile kt-1: wait for that PV's completion.
+          if (!c.wait_warp(B_PVDONE, (tcount - 1) & 1)) return;
+          tc_fence_after();
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t rr[32];
-          tmem_ld32(tO + cc * 32, rr);
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t rr[32];
+            tmem_ld32(tO + cc * 32, rr);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * a);
-          tmem_st32(tO + cc * 32, rr);
+            for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
+            tmem_st32(tO + cc * 32, rr);
+          }
         }
+        l_tile = exp_tile(s, sc, m_run == -INFINITY ? 0.f : -m_run, w);
       }
-      // exponentials (MUFU ex2), row sum in 8 independent chains, P (bf16
-      // pairs) into TMEM over S
-      float ls[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {               // 2 x 32 columns = 128 keys
-        uint32_t w[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float x0 = fmaf(s[cc * 64 + 2 * j], p.scale_log2, neg);
-          const float x1 = fmaf(s[cc * 64 + 2 * j + 1], p.scale_log2, neg);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          ls[j & 7] += p0 + p1;
-          w[j] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + cc * 32, w);
-      }
-      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      l_run += l_tile;
+      tmem_st32(tS, w);
+      tmem_st32(tS + 32, w + 32);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(c.bar(B_PFULL_A + X));
+      mbar_arrive(c.bar(B_PFULL0 + sb));
     }
+    // Hand the row's normaliser to the epilogue warpgroup.  The slot was last
+    // used by unit uc-2: wait until the epilogue has released it (a unit of
+    // one or two key tiles can otherwise get here before that epilogue ran).
+    if (!c.wait_warp(B_OEMPTY0 + (uc & 1), ((uc >> 1) & 1) ^ 1)) return;
+    inv_l[128 * (uc & 1) + r] = l_run > 0.f ? 1.f / l_run : 0.f;
+    mbar_arrive(c.bar(B_LFULL0 + (uc & 1)));
+    ++uc;
+  }
+}
 
-    // epilogue: O / l -> bf16 -> global
-    if (!c.wait(B_OFULL_A + X, o_cnt & 1)) return;
-    ++o_cnt;
+// ---------------------------------------------------------------------------
+// Epilogue role: 128 threads write the unit's 128 output rows.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void epilogue_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
+                                              const float* inv_l, int warp, int lane) {
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+  uint32_t uc = 0;
+  for (uint32_t i = 0;; ++i) {
+    int u;
+    if (!c.next_unit(i, lane, true, &u)) return;
+    if (u >= p.n_units) return;
+    const UnitInfo x = decode_unit(p, u);
+    const uint32_t ob = uc & 1;
+    if (!c.wait_warp(B_OFULL0 + ob, (uc >> 1) & 1)) return;
+    if (!c.wait_warp(B_LFULL0 + ob, (uc >> 1) & 1)) return;
     tc_fence_after();
-    __syncwarp();
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    const uint32_t tO = tmem + lane_base + kColO + 128u * ob;
+    const float inv = inv_l[128 * ob + r];
+    const int i_row = x.m * 128 + r;
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)x.zq * p.N + (size_t)i_row) * kD;
     const bool store = i_row < p.N;
 #pragma unroll 1
@@ -296,103 +361,65 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
       }
     }
     tc_fence_before();
-    mbar_arrive(c.bar(B_OEMPTY_A + X));
+    mbar_arrive(c.bar(B_OEMPTY0 + ob));
+    ++uc;
   }
 }
 
 // ---------------------------------------------------------------------------
 // MMA role: one thread.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint32_t sV, bool first) {
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_bf16_ts(tO, tP + (uint32_t)kk * 8u, desc_v(sV, kk), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-}
-
 __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
                                          uint32_t sQ0, uint32_t sK0, uint32_t sV0) {
-  Ring kr, vr;                              // K and V ring positions
-  uint32_t qc = 0;                          // units consumed
-  uint32_t pc[2] = {0, 0}, oe[2] = {0, 0};  // P tiles consumed, units started per X
+  Ring kr, vr;                      // K and V ring positions
+  uint32_t tc = 0, tp = 0, uc = 0;  // S tiles issued, PV tiles issued, units
   for (uint32_t i = 0;; ++i) {
-    if (!c.wait(B_UFULL0 + (i & 1), (i >> 1) & 1)) return;
-    const int u = c.ring[i & 1];
-    mbar_arrive(c.bar(B_UEMPTY0 + (i & 1)));
+    int u;
+    if (!c.next_unit(i, 0, false, &u)) return;
     if (u >= p.n_units) return;
     const UnitInfo x = decode_unit(p, u);
-    const int lo = x.loA;
-    const int hi = x.actB ? x.hiB : x.hiA;
-    if (!c.wait(B_QFULL, qc & 1)) return;
-    ++qc;
+    const uint32_t ob = uc & 1;
+    const uint32_t tO = tmem + kColO + 128u * ob;
+    const uint32_t sQ = sQ0 + ob * kTileBytes;
+    if (!c.wait(B_QFULL0 + ob, (uc >> 1) & 1)) return;
     tc_fence_after();
-    bool first_pv[2] = {true, true};
-    uint32_t v_prev = 0;                   // V stage of key tile kt-1
-    for (int kt = lo; kt <= hi; ++kt) {
-      const uint32_t ks = kr.stage;
-      if (!c.wait(B_KFULL0 + ks, kr.phase)) return;
+    // PV of the unit's tile jj (P in the S buffer that tile used).
+    auto pv = [&](bool first) -> bool {
+      if (!c.wait(B_PFULL0 + (tp & 1), (tp >> 1) & 1)) return false;
+      if (!c.wait(B_VFULL0 + vr.stage, vr.phase)) return false;
+      if (first && !c.wait(B_OEMPTY0 + ob, ((uc >> 1) & 1) ^ 1)) return false;
+      tc_fence_after();
+      const uint32_t tP = tmem + kColS + 128u * (tp & 1);
+      const uint32_t sV = sV0 + vr.stage * kTileBytes;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ts(tO, tP + (uint32_t)kk * 8u, desc_v(sV, kk), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+      mma_commit(c.bar(B_PVDONE));
+      mma_commit(c.bar(B_VEMPTY0 + vr.stage));
+      vr.next(kVStages);
+      ++tp;
+      return true;
+    };
+    for (int kt = x.lo; kt <= x.m; ++kt) {
+      // S(kt) = Q K(kt)^T into S buffer tc & 1
+      if (!c.wait(B_KFULL0 + kr.stage, kr.phase)) return;
+      tc_fence_after();
+      const uint32_t sK = sK0 + kr.stage * kTileBytes;
+      const uint32_t tS = tmem + kColS + 128u * (tc & 1);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tS, desc_kmajor(sQ, kk), desc_kmajor(sK, kk), IDESC_QK, kk > 0 ? 1u : 0u);
+      mma_commit(c.bar(B_SFULL0 + (tc & 1)));
+      mma_commit(c.bar(B_KEMPTY0 + kr.stage));
       kr.next(kKStages);
-      tc_fence_after();
-      if (kt > lo) {                       // V(kt-1) feeds this step's PVs
-        v_prev = vr.stage;
-        if (!c.wait(B_VFULL0 + v_prev, vr.phase)) return;
-        vr.next(kVStages);
-        tc_fence_after();
-      }
-#pragma unroll
-      for (int X = 0; X < 2; ++X) {
-        const bool act = X == 0 || x.actB;
-        const int loX = X == 0 ? x.loA : x.loB;
-        const int hiX = X == 0 ? x.hiA : x.hiB;
-        if (!act) continue;
-        if (kt - 1 >= loX && kt - 1 <= hiX) {                // O_X += P_X(kt-1) V(kt-1)
-          if (!c.wait(B_PFULL_A + X, pc[X] & 1)) return;
-          ++pc[X];
-          if (first_pv[X]) {
-            if (!c.wait(B_OEMPTY_A + X, (oe[X] & 1) ^ 1)) return;
-            ++oe[X];
-          }
-          tc_fence_after();
-          issue_pv(tmem + 256u + 128u * X, tmem + 128u * X, sV0 + v_prev * kTileBytes, first_pv[X]);
-          first_pv[X] = false;
-        }
-        if (kt >= loX && kt <= hiX) {                        // S_X = Q_X K(kt)^T
-          const uint32_t sK = sK0 + ks * kTileBytes;
-          const uint32_t sQ = sQ0 + (uint32_t)X * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ss(tmem + 128u * X, desc_kmajor(sQ, kk), desc_kmajor(sK, kk), IDESC_QK,
-                        kk > 0 ? 1u : 0u);
-          mma_commit(c.bar(B_SFULL_A + X));
-        }
-      }
-      mma_commit(c.bar(B_KEMPTY0 + ks));
-      if (kt > lo) mma_commit(c.bar(B_VEMPTY0 + v_prev));
+      ++tc;
+      if (kt == x.m) mma_commit(c.bar(B_QEMPTY0 + ob));   // every S of the unit issued
+      // O += P(kt-1) V(kt-1)
+      if (kt > x.lo && !pv(kt - 1 == x.lo)) return;
     }
-    mma_commit(c.bar(B_QEMPTY));           // every S of the unit is issued
-    // tail: PVs of the last key tile
-    v_prev = vr.stage;
-    if (!c.wait(B_VFULL0 + v_prev, vr.phase)) return;
-    vr.next(kVStages);
-    tc_fence_after();
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      const bool act = X == 0 || x.actB;
-      const int loX = X == 0 ? x.loA : x.loB;
-      const int hiX = X == 0 ? x.hiA : x.hiB;
-      if (!act || hi < loX || hi > hiX) continue;
-      if (!c.wait(B_PFULL_A + X, pc[X] & 1)) return;
-      ++pc[X];
-      if (first_pv[X]) {
-        if (!c.wait(B_OEMPTY_A + X, (oe[X] & 1) ^ 1)) return;
-        ++oe[X];
-      }
-      tc_fence_after();
-      issue_pv(tmem + 256u + 128u * X, tmem + 128u * X, sV0 + v_prev * kTileBytes, first_pv[X]);
-      first_pv[X] = false;
-    }
-    mma_commit(c.bar(B_VEMPTY0 + v_prev));
-    mma_commit(c.bar(B_OFULL_A));
-    if (x.actB) mma_commit(c.bar(B_OFULL_B));
+    if (!pv(x.m == x.lo)) return;                   // last tile's PV
+    mma_commit(c.bar(B_OFULL0 + ob));
+    ++uc;
   }
 }
 
@@ -412,18 +439,14 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
     mbar_arrive(c.bar(B_UFULL0 + (i & 1)));
     if (u >= p.n_units) return;
     const UnitInfo x = decode_unit(p, u);
-    const int lo = x.loA;
-    const int hi = x.actB ? x.hiB : x.hiA;
-    if (!c.wait(B_QEMPTY, (qc & 1) ^ 1)) return;
+    const uint32_t qb = qc & 1;
+    if (!c.wait(B_QEMPTY0 + qb, ((qc >> 1) & 1) ^ 1)) return;
     ++qc;
-    mbar_expect_tx(c.bar(B_QFULL), x.actB ? 2 * kTileBytes : kTileBytes);
-    tma_load_3d(sQ0, tmQ, c.bar(B_QFULL), 0, x.hiA * 128, x.zq);
-    tma_load_3d(sQ0 + kHalfBytes, tmQ, c.bar(B_QFULL), 64, x.hiA * 128, x.zq);
-    if (x.actB) {
-      tma_load_3d(sQ0 + kTileBytes, tmQ, c.bar(B_QFULL), 0, x.hiB * 128, x.zq);
-      tma_load_3d(sQ0 + kTileBytes + kHalfBytes, tmQ, c.bar(B_QFULL), 64, x.hiB * 128, x.zq);
-    }
-    for (int kt = lo; kt <= hi; ++kt) {
+    const uint32_t sQ = sQ0 + qb * kTileBytes;
+    mbar_expect_tx(c.bar(B_QFULL0 + qb), kTileBytes);
+    tma_load_3d(sQ, tmQ, c.bar(B_QFULL0 + qb), 0, x.m * 128, x.zq);
+    tma_load_3d(sQ + kHalfBytes, tmQ, c.bar(B_QFULL0 + qb), 64, x.m * 128, x.zq);
+    for (int kt = x.lo; kt <= x.m; ++kt) {
       const uint32_t ks = kr.stage;
       if (!c.wait(B_KEMPTY0 + ks, kr.phase ^ 1)) return;
       kr.next(kKStages);
@@ -457,12 +480,15 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   c.ring = reinterpret_cast<volatile int*>(smem + OFF_UNIT);
   c.hdr = p.hdr;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
+  float* inv_l = reinterpret_cast<float*>(smem + OFF_INVL);
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PFULL_A || i == B_PFULL_B || i == B_OEMPTY_A || i == B_OEMPTY_B) cnt = 128;
-      if (i == B_UEMPTY0 || i == B_UEMPTY1) cnt = 9;   // MMA thread + 8 softmax warps
+      if (i == B_PFULL0 || i == B_PFULL1 || i == B_LFULL0 || i == B_LFULL1 || i == B_OEMPTY0 ||
+          i == B_OEMPTY1)
+        cnt = 128;
+      if (i == B_UEMPTY0 || i == B_UEMPTY1) cnt = 9;   // MMA thread + 4 softmax + 4 epilogue warps
       mbar_init(c.bar(i), cnt);
     }
     *c.abort = 0;
@@ -480,12 +506,15 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp < 4) {
     regs_dec<kRegsControl>();
     if (warp == 0 && lane == 0)
-      producer_role(p, c, &tmQ, &tmK, &tmV, sbase + OFF_QA, sbase + OFF_K, sbase + OFF_V);
+      producer_role(p, c, &tmQ, &tmK, &tmV, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
     else if (warp == 1 && lane == 0)
-      mma_role(p, c, tmem, sbase + OFF_QA, sbase + OFF_K, sbase + OFF_V);
-  } else {
+      mma_role(p, c, tmem, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
+  } else if (warp < 8) {
     regs_inc<kRegsSoftmax>();
-    softmax_role(p, c, tmem, warp < 8 ? 0 : 1, warp, lane);
+    softmax_role(p, c, tmem, inv_l, warp, lane);
+  } else {
+    regs_dec<kRegsEpilogue>();
+    epilogue_role(p, c, tmem, inv_l, warp, lane);
   }
 
   // teardown: after a timeout give in-flight copies and MMAs time to land
@@ -537,46 +566,32 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 
 }  // namespace
 
-// Units of two query tiles (256 rows); a unit's cost is the number of
-// (query tile, key tile) pairs it visits.
+// Units of one 128-row query tile; a unit's cost is its number of key tiles.
 std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans) {
   const int64_t M = (N + kTileM - 1) / kTileM;      // query tiles
-  const int64_t MP = (M + 1) / 2;                   // units per head
-  struct U { int32_t b, h, mp; int64_t cost; };
+  struct U { int32_t b, h, m, lo; int64_t cost; };
   std::vector<U> v;
-  v.reserve((size_t)B * Hq * MP);
+  v.reserve((size_t)B * Hq * M);
   for (int32_t b = 0; b < B; ++b)
     for (int32_t h = 0; h < Hq; ++h)
-      for (int64_t mp = 0; mp < MP; ++mp) {
-        const int64_t qa = 2 * mp, qb = 2 * mp + 1;
-        int64_t cost = qa - first_tile_host(qa, spans[h]) + 1;
-        if (qb < M) cost += qb - first_tile_host(qb, spans[h]) + 1;
-        v.push_back({b, h, (int32_t)mp, cost});
+      for (int64_t m = 0; m < M; ++m) {
+        const int64_t lo = first_tile_host(m, spans[h]);
+        v.push_back({b, h, (int32_t)m, (int32_t)lo, m - lo + 1});
       }
   std::stable_sort(v.begin(), v.end(), [](const U& a, const U& c) { return a.cost > c.cost; });
   std::vector<int32_t> out(v.size() * 4);
   for (size_t i = 0; i < v.size(); ++i) {
     out[4 * i + 0] = v[i].b;
     out[4 * i + 1] = v[i].h;
-    out[4 * i + 2] = v[i].mp;
-    out[4 * i + 3] = 0;
+    out[4 * i + 2] = v[i].m;
+    out[4 * i + 3] = v[i].lo;
   }
   return out;
 }
 
-void prefill_unit_tiles(int32_t N, int32_t S, int32_t mp, int32_t tiles[4]) {
-  const int64_t M = (N + kTileM - 1) / kTileM;
-  const int64_t qa = 2 * (int64_t)mp, qb = qa + 1;
-  tiles[0] = (int32_t)first_tile_host(qa, S);
-  tiles[1] = (int32_t)qa;
-  tiles[2] = qb < M ? (int32_t)first_tile_host(qb, S) : -1;
-  tiles[3] = qb < M ? (int32_t)qb : -1;
-}
-
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
   const int64_t M = (N + kTileM - 1) / kTileM;
-  const int64_t MP = (M + 1) / 2;
-  return kUnitsOffset + (size_t)B * Hq * MP * 16;
+  return kUnitsOffset + (size_t)B * Hq * M * 16;
 }
 
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
@@ -607,7 +622,6 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
-  p.n_qtiles = (N + kTileM - 1) / kTileM;
   p.scale_log2 = scale * 1.4426950408889634f;
   for (int h = 0; h < Hq; ++h) p.span[h] = spans[h];
 

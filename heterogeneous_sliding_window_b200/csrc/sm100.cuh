@@ -109,6 +109,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr)
       : "memory");
 }
+// Same for 64 consecutive columns in one instruction (one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
 // Same for 128 consecutive columns in one instruction (one wait).
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t* r) {
   asm volatile(
@@ -211,12 +220,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 126 (inputs below -125 give 2^-125).
+// 2^x on the FMA pipe for x in [-125, 64]; inputs outside are clamped to that
+// range (so a huge x gives 2^64 rather than wrapping the exponent field).
 // x = n + f with n = round(x) taken from the low mantissa bits of x + 1.5*2^23
 // and f in [-1/2, 1/2]; 2^f by a cubic fitted to minimax relative error
 // (1.1e-4, see fit_exp2_poly.py); 2^n added into the exponent field.
 __device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
+  x = fminf(fmaxf(x, -125.f), 64.f);
   const float magic = 12582912.f;                 // 1.5 * 2^23
   const float t = x + magic;
   const float n = t - magic;
@@ -225,6 +235,51 @@ __device__ __forceinline__ float exp2_poly(float x) {
   p = fmaf(f, p, 6.932604313e-01f);
   p = fmaf(f, p, 1.0f);
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// ---- packed fp32 pairs (f32x2 arithmetic on a 64-bit register pair) --------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe: the clamp, reduction and cubic of exp2_poly
+// in packed f32x2 arithmetic, then 2^n added into each exponent field.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fminf(fmaxf(a, -125.f), 64.f), fminf(fmaxf(b, -125.f), 64.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);     // 1.5 * 2^23
+  const uint64_t t = f2_add(x2, magic);
+  const uint64_t n = f2_sub(t, magic);
+  const uint64_t f = f2_sub(x2, n);
+  uint64_t q = f2_fma(f, f2_pack(5.511890724e-02f, 5.511890724e-02f), f2_pack(2.422108501e-01f, 2.422108501e-01f));
+  q = f2_fma(f, q, f2_pack(6.932604313e-01f, 6.932604313e-01f));
+  q = f2_fma(f, q, f2_pack(1.0f, 1.0f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -168,12 +168,12 @@ moa_status moa_prefill(const void* q, const void* k, const void* v, void* o,
                        void* workspace, size_t ws_bytes, moa_kv_cache* fill_or_null,
                        void* stream);
 
-/* Host view of the prefill schedule.  The kernel's work unit is two adjacent
- * query tiles of 128 rows of one (sequence, head); units run longest first.
- * One row of 6 int32 per query tile, in the order the persistent kernel takes
- * the units: (unit, b, h, m, lo, hi) -- query rows [128m, 128m+127] visit key
- * tiles lo..hi of 128 keys (hi = m, the diagonal tile).  Writes min(cap, n)
- * rows, *n_rows_out = n.  Host only. */
+/* Host view of the prefill schedule.  The kernel's work unit is one query
+ * tile of 128 rows of one (sequence, head); units run longest first.  One row
+ * of 6 int32 per unit, in the order the persistent kernel takes them:
+ * (unit, b, h, m, lo, hi) -- query rows [128m, 128m+127] visit key tiles
+ * lo..hi of 128 keys (hi = m, the diagonal tile).  Writes min(cap, n) rows,
+ * *n_rows_out = n.  Host only. */
 moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
                                 int32_t* rows_out, int64_t cap, int64_t* n_rows_out);
 

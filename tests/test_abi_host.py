@@ -163,7 +163,7 @@ def test_workspace_sizes():
     d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)
     p = moa.moa_workspace_bytes(moa.MOA_OP_PREFILL, 2, 4, 1000, 128, spans)
     assert d % 256 == 0 and d >= 256 + 2 * 4 * 4
-    assert p >= 256 + 2 * 4 * 4 * 16   # units of two 128-row query tiles
+    assert p >= 256 + 2 * 4 * 8 * 16   # one unit per 128-row query tile
     with pytest.raises(moa.MoaError):
         moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, [64, 0, 1, 1])
 

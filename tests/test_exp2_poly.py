@@ -18,7 +18,7 @@ HDR = os.path.join(ROOT, "heterogeneous_sliding_window_b200", "csrc", "sm100.cuh
 
 def _coefficients():
     text = open(HDR).read()
-    body = text[text.index("float exp2_poly("):]
+    body = text[text.index("float exp2_poly(float x)"):]
     body = body[:body.index("return")]
     nums = [float(x) for x in re.findall(r"fmaf\(f, (?:p|[-0-9.e+]+f), ([-0-9.e+]+)f\)", body)]
     c3 = float(re.search(r"fmaf\(f, ([-0-9.e+]+)f,", body).group(1))
@@ -32,7 +32,7 @@ def _fma32(a, b, c):
 
 def exp2_poly_replay(x):
     c3, c2, c1, c0 = _coefficients()
-    x = np.maximum(x.astype(np.float32), np.float32(-125.0))
+    x = np.minimum(np.maximum(x.astype(np.float32), np.float32(-125.0)), np.float32(64.0))
     magic = np.float32(12582912.0)
     t = (x + magic).astype(np.float32)
     n = (t - magic).astype(np.float32)
@@ -65,3 +65,5 @@ def test_exp2_poly_integers_and_clamp():
         assert abs(v / 2.0 ** n - 1.0) < 2e-4
     tiny = exp2_poly_replay(np.array([-np.inf, -1e30, -200.0], dtype=np.float32))
     assert np.all(tiny > 0) and np.all(tiny < 3e-38)
+    huge = exp2_poly_replay(np.array([np.inf, 1e30, 500.0, 64.0], dtype=np.float32))
+    assert np.all(np.abs(huge / 2.0 ** 64 - 1.0) < 2e-4)      # clamped, never wrapped

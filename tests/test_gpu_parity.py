@@ -108,6 +108,24 @@ def test_bf16_prefill_matches_oracle(case):
     assert err <= BF16_TOL, err
 
 
+def test_bf16_prefill_scores_growing_along_the_sequence():
+    """Key norms grow with position, so later tiles' maxima jump far above the
+    running maximum (the kernel's rescale path) and early tiles underflow."""
+    B, Hq, N, d = 1, 4, 900, 128
+    spans = [900, 300, 129, 640]
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn(31, (B, Hq, N, d), "f32")
+    k = inputs.randn(32, (B, Hq, N, d), "f32")
+    growth = torch.linspace(0.2, 12.0, N).view(1, 1, N, 1)
+    k = (k * growth).to(torch.bfloat16)
+    q = (q * 2.0).to(torch.bfloat16)
+    v = inputs.randn(33, (B, Hq, N, d))
+    o = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, scale)
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale)
+    err = np.max(np.abs(inputs.as_f64(o) - ref))
+    assert err <= BF16_TOL, err
+
+
 def test_bf16_prefill_fill_cache_bytes():
     B, Hq, Hkv, N, d = 2, 4, 2, 600, 128
     spans = [64, 256, 600, 100]
