@@ -6,14 +6,18 @@
 // HBM-bound: every cached key and value of the window is read once.
 //
 // Grid: one CTA per (sequence b, head h, split s) where split s covers window
-// entries [s*kChunk, (s+1)*kChunk).  A CTA
-//   1. streams its K rows with 16-byte loads (a row is spread over LPR lanes),
-//      forms q.k in fp32 and reduces each dot product with xor-shuffles;
-//   2. takes the chunk max m and p_j = 2^(s_j - m), l = sum p_j;
-//   3. streams its V rows and accumulates sum p_j v_j in fp32;
-//   4. single split: writes o = acc / l.  Otherwise writes (m, l, acc) to the
-//      workspace; the last split of (b, h) to finish (atomic ticket) merges all
-//      partials with the log-sum-exp rule and writes o, then rearms its ticket.
+// entries [s*kChunk, (s+1)*kChunk).  The CTA's 128 threads form row groups of
+// LPR lanes (one 16-byte vector of a cached row per lane); each group walks
+// its share of the chunk in batches of kUnroll rows, issuing the K and V loads
+// of a whole batch together (2*kUnroll 16-byte loads in flight per thread),
+// and keeps an online softmax (running max m, sum l, fp32 accumulator) over
+// its rows:
+//   s_j = scale * q.k_j (xor-shuffle reduction over the group's lanes)
+//   m' = max(m, s_j over the batch), acc = acc * 2^(m - m') + sum p_j v_j
+// The groups then merge in shared memory with the log-sum-exp rule.  A single
+// split writes o = acc / l; otherwise the CTA writes (m, l, acc) to the
+// workspace and the last split of (b, h) to finish (atomic ticket) merges all
+// partials the same way, writes o, and rearms its ticket.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -23,8 +27,8 @@ namespace {
 
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kChunk = 256;          // window entries per split
-constexpr int kUnroll = 4;           // independent 16-byte loads in flight per thread
+constexpr int kChunk = 512;          // window entries per split
+constexpr int kUnroll = 8;           // rows per batch: 2*kUnroll 16-byte loads in flight
 
 struct DecodeParams {
   const char* data;                  // cache data region
@@ -66,33 +70,22 @@ template <> struct Vec16<__nv_bfloat16> {
   __device__ static void store(__nv_bfloat16* dst, float x) { *dst = __float2bfloat16_rn(x); }
 };
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int VE = Vec16<T>::N;     // elements per 16-byte vector
   constexpr int LPR = D / VE;         // lanes per cached row
-  constexpr int RPW = 32 / LPR;       // rows per warp per step
-  constexpr int RPS = RPW * kDecWarps;
+  constexpr int RPW = 32 / LPR;       // row groups per warp
+  constexpr int NG = RPW * kDecWarps; // row groups per CTA
   static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row must map onto a warp");
 
-  __shared__ float sc[kChunk];
-  __shared__ float red[RPS][D];
-  __shared__ float wred[kDecWarps];
+  __shared__ float g_acc[NG][D];
+  __shared__ float g_m[NG], g_l[NG];
   __shared__ int last_flag;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int sub = lane / LPR, li = lane % LPR;
+  const int grp = warp * RPW + sub;
 
   const int item = blockIdx.x;
   const int b = item / p.items_per_b;
@@ -126,105 +119,95 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
     for (int e = 0; e < VE; ++e) qf[e] *= p.scale_log2;
   }
 
-  // Phase 1: scores (log2 domain).
-  for (int base = 0; base < nrows; base += RPS * kUnroll) {
-    int4 raw[kUnroll];
+  float m = -INFINITY, l = 0.f;
+  float acc[VE];
+#pragma unroll
+  for (int e = 0; e < VE; ++e) acc[e] = 0.f;
+
+  // The trip count is uniform across the CTA (every lane takes part in the
+  // shuffles below); rows past the chunk are masked instead.
+  for (int base = 0; base < nrows; base += NG * kUnroll) {
+    int4 kr[kUnroll], vr[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int row = base + u * RPS + warp * RPW + sub;
+      const int row = base + u * NG + grp;
       if (row < nrows) {
         int slot = slot0 + row;
         if (slot >= C) slot -= C;
-        raw[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
+        kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
+        vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
       } else {
-        raw[u] = make_int4(0, 0, 0, 0);
+        kr[u] = make_int4(0, 0, 0, 0);
+        vr[u] = make_int4(0, 0, 0, 0);
       }
     }
+    float sv[kUnroll];
+    float bmax = m;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       float kf[VE];
-      Vec16<T>::cvt(raw[u], kf);
+      Vec16<T>::cvt(kr[u], kf);
       float dot = 0.f;
 #pragma unroll
       for (int e = 0; e < VE; ++e) dot = fmaf(qf[e], kf[e], dot);
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      const int row = base + u * RPS + warp * RPW + sub;
-      if (li == 0 && row < nrows) sc[row] = dot;
+      sv[u] = (base + u * NG + grp < nrows) ? dot : -INFINITY;
+      bmax = fmaxf(bmax, sv[u]);
     }
-  }
-  __syncthreads();
-
-  // Phase 2: chunk max and exponentials.
-  float m = -INFINITY;
-  for (int i = tid; i < nrows; i += kDecThreads) m = fmaxf(m, sc[i]);
-  m = warp_max(m);
-  if (lane == 0) wred[warp] = m;
-  __syncthreads();
-  m = wred[0];
+    if (bmax > m) {                                   // uniform across the group's lanes
+      const float corr = exp2f(m - bmax);             // 0 when m = -inf
+      l *= corr;
 #pragma unroll
-  for (int w = 1; w < kDecWarps; ++w) m = fmaxf(m, wred[w]);
-  __syncthreads();
-  float l = 0.f;
-  for (int i = tid; i < nrows; i += kDecThreads) {
-    const float e = exp2f(sc[i] - m);
-    sc[i] = e;
-    l += e;
-  }
-  l = warp_sum(l);
-  if (lane == 0) wred[warp] = l;
-  __syncthreads();
-  l = 0.f;
-#pragma unroll
-  for (int w = 0; w < kDecWarps; ++w) l += wred[w];
-
-  // Phase 3: weighted sum of values.
-  float acc[VE];
-#pragma unroll
-  for (int e = 0; e < VE; ++e) acc[e] = 0.f;
-  for (int base = 0; base < nrows; base += RPS * kUnroll) {
-    int4 raw[kUnroll];
+      for (int e = 0; e < VE; ++e) acc[e] *= corr;
+      m = bmax;
+    }
+    // A group that has seen no row yet keeps m = -inf; its masked scores must
+    // still give p = 0, not 2^(-inf - -inf) = NaN.
+    const float mref = m == -INFINITY ? 0.f : m;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int row = base + u * RPS + warp * RPW + sub;
-      if (row < nrows) {
-        int slot = slot0 + row;
-        if (slot >= C) slot -= C;
-        raw[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
-      } else {
-        raw[u] = make_int4(0, 0, 0, 0);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int row = base + u * RPS + warp * RPW + sub;
-      const float pr = row < nrows ? sc[row] : 0.f;
+      const float pu = exp2f(sv[u] - mref);           // 0 for rows past the chunk
+      l += pu;
       float vf[VE];
-      Vec16<T>::cvt(raw[u], vf);
+      Vec16<T>::cvt(vr[u], vf);
 #pragma unroll
-      for (int e = 0; e < VE; ++e) acc[e] = fmaf(pr, vf[e], acc[e]);
+      for (int e = 0; e < VE; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
     }
   }
+
+  // merge the row groups (log-sum-exp)
 #pragma unroll
-  for (int e = 0; e < VE; ++e) red[warp * RPW + sub][li * VE + e] = acc[e];
+  for (int e = 0; e < VE; ++e) g_acc[grp][li * VE + e] = acc[e];
+  if (li == 0) {
+    g_m[grp] = m;
+    g_l[grp] = l;
+  }
   __syncthreads();
-  float od = 0.f;
-  if (tid < D) {
+  float M = -INFINITY;
 #pragma unroll
-    for (int rr = 0; rr < RPS; ++rr) od += red[rr][tid];
+  for (int k = 0; k < NG; ++k) M = fmaxf(M, g_m[k]);
+  float L = 0.f, od = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+      const float w = exp2f(g_m[k] - M);
+      L = fmaf(w, g_l[k], L);
+      if (tid < D) od = fmaf(w, g_acc[k][tid], od);
+    }
   }
 
   T* out = reinterpret_cast<T*>(p.o) + ((size_t)b * p.Hq + h) * D;
   if (nsplit == 1) {
-    if (tid < D) Vec16<T>::store(out + tid, l > 0.f ? od / l : 0.f);
+    if (tid < D) Vec16<T>::store(out + tid, L > 0.f ? od / L : 0.f);
     if (tid == 0 && Seff == 0) atomicOr(p.err, kErrEmpty);
     return;
   }
   const size_t idx = (size_t)b * p.items_per_b + r;
   if (tid < D) p.part_o[idx * D + tid] = od;
   if (tid == 0) {
-    p.part_ml[2 * idx] = m;
-    p.part_ml[2 * idx + 1] = l;
+    p.part_ml[2 * idx] = M;
+    p.part_ml[2 * idx + 1] = L;
   }
   __threadfence();
   __syncthreads();
@@ -236,22 +219,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   if (!last_flag) return;
   __threadfence();
   const size_t first = (size_t)b * p.items_per_b + p.split_pre[h];
-  float M = -INFINITY;
-  for (int ss = 0; ss < nsplit; ++ss) M = fmaxf(M, __ldcg(&p.part_ml[2 * (first + ss)]));
-  float L = 0.f, A = 0.f;
-  if (M != -INFINITY) {
+  float MM = -INFINITY;
+  for (int ss = 0; ss < nsplit; ++ss) MM = fmaxf(MM, __ldcg(&p.part_ml[2 * (first + ss)]));
+  float LL = 0.f, A = 0.f;
+  if (MM != -INFINITY) {
     for (int ss = 0; ss < nsplit; ++ss) {
       const float ms = __ldcg(&p.part_ml[2 * (first + ss)]);
-      const float w = exp2f(ms - M);              // 0 for empty splits (ms = -inf)
-      L = fmaf(w, __ldcg(&p.part_ml[2 * (first + ss) + 1]), L);
+      const float w = exp2f(ms - MM);              // 0 for empty splits (ms = -inf)
+      LL = fmaf(w, __ldcg(&p.part_ml[2 * (first + ss) + 1]), LL);
       if (tid < D) A = fmaf(w, __ldcg(&p.part_o[(first + ss) * D + tid]), A);
     }
   }
-  if (tid < D) Vec16<T>::store(out + tid, L > 0.f ? A / L : 0.f);
+  if (tid < D) Vec16<T>::store(out + tid, LL > 0.f ? A / LL : 0.f);
   if (tid == 0) {
     p.ctr[(size_t)b * p.Hq + h] = 0u;
     if (Seff == 0) atomicOr(p.err, kErrEmpty);
   }
+}
+
+template <typename T, int D>
+cudaError_t launch_one(const DecodeParams& p, unsigned grid, cudaStream_t s) {
+  decode_kernel<T, D><<<grid, kDecThreads, 0, s>>>(p);
+  return cudaGetLastError();
 }
 
 struct DecodeLayout {
@@ -308,14 +297,13 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   }
   const long long grid = (long long)c->B * L.items_per_b;
   if (grid > 0x7fffffffLL) return MOA_ERR_UNSUPPORTED;
-  if (c->dtype == MOA_BF16) {
-    if (c->d == 128) decode_kernel<__nv_bfloat16, 128><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
-    else decode_kernel<__nv_bfloat16, 64><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
-  } else {
-    if (c->d == 128) decode_kernel<float, 128><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
-    else decode_kernel<float, 64><<<(unsigned)grid, kDecThreads, 0, s>>>(p);
-  }
-  return check_launch("decode launch");
+  cudaError_t e;
+  if (c->dtype == MOA_BF16)
+    e = c->d == 128 ? launch_one<__nv_bfloat16, 128>(p, (unsigned)grid, s)
+                    : launch_one<__nv_bfloat16, 64>(p, (unsigned)grid, s);
+  else
+    e = c->d == 128 ? launch_one<float, 128>(p, (unsigned)grid, s) : launch_one<float, 64>(p, (unsigned)grid, s);
+  return e == cudaSuccess ? MOA_OK : cuda_fail(e, "decode launch");
 }
 
 }  // namespace moa
