@@ -1,6 +1,7 @@
 // C ABI front end of libmoa: argument validation and dispatch to the kernels.
 // Every check that can fail does so here, on the host, before anything is
 // enqueued; the kernels assume validated arguments.
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -173,23 +174,16 @@ extern "C" moa_status moa_workspace_check(const void* ws, void* stream) {
 }
 
 extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
-                                           int32_t* rows_out, int64_t cap, int64_t* n_rows_out) {
+                                           int32_t n_ctas, int32_t* rows_out, int64_t cap,
+                                           int64_t* n_rows_out) {
   if (B < 1 || Hq < 1 || Hq > MOA_MAX_HEADS || N < 1 || N > INT32_MAX || !spans || !n_rows_out ||
-      cap < 0 || (cap > 0 && !rows_out))
+      n_ctas < 1 || n_ctas > kPrefillMaxCtas || cap < 0 || (cap > 0 && !rows_out))
     return MOA_ERR_INVALID_ARG;
   for (int32_t h = 0; h < Hq; ++h)
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
-  std::vector<int32_t> u = prefill_units(B, Hq, (int32_t)N, spans);
-  const int64_t n = (int64_t)u.size() / 4;
-  for (int64_t i = 0; i < n && i < cap; ++i) {
-    int32_t* r = rows_out + 6 * i;
-    r[0] = (int32_t)i;
-    r[1] = u[4 * i];
-    r[2] = u[4 * i + 1];
-    r[3] = u[4 * i + 2];   // query tile m
-    r[4] = u[4 * i + 3];   // lo
-    r[5] = u[4 * i + 2];   // hi: the diagonal tile
-  }
+  const std::vector<int32_t> rows = prefill_schedule_rows(B, Hq, (int32_t)N, spans, n_ctas);
+  const int64_t n = (int64_t)rows.size() / 7;
+  std::copy(rows.begin(), rows.begin() + 7 * std::min(n, cap), rows_out);
   *n_rows_out = n;
   return MOA_OK;
 }

@@ -62,9 +62,20 @@ moa_status launch_prefill_f32(const float* q, const float* k, const float* v, fl
                               const int32_t* spans, float scale, cudaStream_t s);
 
 // prefill_sm100.cu (bf16, tcgen05)
-constexpr int kTileM = 128;   // query rows per work unit
+constexpr int kTileM = 128;   // query rows per query tile (a work unit holds two)
 constexpr int kTileN = 128;   // keys per key/value tile
-std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans);
+constexpr int kPrefillMaxCtas = 1024;   // persistent grid bound (one CTA per SM)
+// Work units (b, h, first query tile m, first key tile of m), dealt to n_ctas
+// per-CTA lists: CTA c runs units[off[c] .. off[c+1]) in order.
+struct PrefillSchedule {
+  int32_t n_ctas;
+  std::vector<int32_t> off;     // n_ctas + 1
+  std::vector<int32_t> units;   // 4 int32 per unit
+};
+PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas);
+// Rows (CTA, unit, b, h, query tile, first key tile, last key tile), one per query tile.
+std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, const int32_t* spans,
+                                           int32_t n_ctas);
 
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,

@@ -6,33 +6,41 @@
 // applied to v_j.  Heads differ only in S_h.
 //
 // How (B200 design, not the pages' A100 kernel):
-//  * Work unit = (b, h, m): query rows [128m, 128m+128) of one head.  Because
-//    the window is a band, the unit needs exactly the key tiles lo..m
-//    (lo = floor(max(0, 128m - S_h + 1) / 128)); every other key tile is
-//    skipped.
-//  * Units are sorted longest-first on the host and handed out by a
-//    persistent grid (one CTA per SM): a producer thread takes the next unit
-//    from an atomic counter and publishes it through a two-slot ring in
-//    shared memory, so heads with very different spans balance across SMs.
-//  * Warp roles (384 threads, setmaxnreg split 144 / 216 / 144):
-//      warp 0       TMA producer: Q once per unit into one of two buffers
-//                   (the next unit's Q loads while this unit runs), K and V
-//                   tiles through two-stage rings (128-byte swizzle).
-//      warp 1       MMA issuer (one thread), tcgen05.mma M=128, N=128, K=16:
-//                   S(k) = Q K(k)^T into one of two S buffers in tensor memory,
-//                   O += P(k-1) V(k-1) with P read from tensor memory.  S(k+1)
-//                   is issued right after PV(k-1), without waiting for the
-//                   softmax of tile k, so the tensor core works on the next
-//                   tile while the current tile's exponentials run.
-//      warps 4-7    softmax: one thread per query row reads its S row, masks
-//                   only tiles that cross the diagonal or the window's lower
-//                   edge, takes exponentials against the row's running maximum
-//                   (exact tile maxima only when needed, see softmax_role),
-//                   and writes P as bf16 pairs back over its S buffer.
-//      warps 8-11   epilogue: O / l -> bf16 (round to nearest even) -> global,
-//                   from one of two O buffers, so the next unit's PVs proceed
-//                   while the previous unit is written out.
-//    Tensor memory: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+//  * Work unit = (b, h, m): query tiles A = m and B = m + 1 (128 rows each)
+//    of one head.  Because the window is a band, tile A needs exactly the
+//    key tiles loA..m and tile B the tiles loB..m+1
+//    (lo = floor(max(0, 128t - S_h + 1) / 128) for query tile t); every other
+//    key tile is skipped, and the two tiles share one stream of K and V tiles
+//    loA..m+1.  A head with an odd number of query tiles ends with a unit
+//    that has tile A only.
+//  * Units are dealt on the host to one list per CTA of the persistent grid
+//    (one CTA per SM), longest first, each to the list with the least work
+//    so far, so heads with very different spans balance across SMs without
+//    atomics and every CTA can read its next units ahead of time.
+//  * Warp roles (384 threads, setmaxnreg split 120 / 192 / 192):
+//      warp 0       TMA producer: the unit's two Q tiles into three rotating
+//                   Q slots (the next unit's Q loads while this unit runs),
+//                   K and V tiles through two-stage rings (128-byte swizzle).
+//      warp 1       MMA issuer (one thread), tcgen05.mma M=128, N=128, K=16.
+//                   Per key tile j:  O_A += P_A(j) V(j),  S_A(j+1) = Q_A K(j+1)^T,
+//                   O_B += P_B(j) V(j),  S_B(j+1) = Q_B K(j+1)^T.
+//                   The tensor core works on one tile's PV and next S while
+//                   the other tile's softmax runs (ping-pong).  Each S-ready
+//                   commit also covers that tile's previous PV.  In a unit's
+//                   last key tile, where only tile B is left, the next unit's
+//                   first S_A is issued, so tile A's softmax starts the next
+//                   unit while tile B finishes this one.
+//      warp 2       unit fetcher: this CTA's unit records into a four-slot
+//                   ring in shared memory.
+//      warps 4-7    softmax of tile A, warps 8-11 softmax of tile B: one
+//                   thread per query row reads its S row in two 64-column
+//                   halves, masks only tiles that cross the diagonal or the
+//                   window's lower edge, takes exponentials against a
+//                   per-row reference (see softmax_role), and writes P as
+//                   bf16 pairs back over S; after the unit's last tile it
+//                   reads O, releases the O buffer, and writes O / l as bf16
+//                   (round to nearest even).
+//    Tensor memory: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 //  * Rows >= N are dropped at the store; out-of-range TMA rows read as zeros.
 //  * Every mbarrier wait is bounded (2 s of globaltimer, or earlier if another
 //    role gave up); on a timeout the kernel sets the workspace error word,
@@ -43,7 +51,9 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <functional>
 #include <mutex>
+#include <queue>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -55,21 +65,20 @@ using namespace sm100;
 
 constexpr int kThreads = 384;                    // 3 warpgroups
 // Register split (setmaxnreg): the block launches with 384 x 168 registers;
-// warpgroup 0 (producer, MMA issuer, two idle warps) and the epilogue
-// warpgroup drop to 144, the softmax warpgroup rises to 216.
-constexpr uint32_t kRegsLaunch = 168, kRegsControl = 144, kRegsSoftmax = 216, kRegsEpilogue = 144;
-static_assert(128 * (kRegsControl + kRegsSoftmax + kRegsEpilogue) <= kThreads * kRegsLaunch,
-              "register split");
+// warpgroup 0 (producer, MMA issuer, unit fetcher, one idle warp) drops to
+// 120, the two softmax warpgroups rise to 192.
+constexpr uint32_t kRegsLaunch = 168, kRegsControl = 120, kRegsSoftmax = 192;
+static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kThreads * kRegsLaunch, "register split");
 constexpr int kD = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one 128 x 128 bf16 tile
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizzled half
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
+constexpr uint32_t kQSlots = 3;                       // rotating Q tiles (two per unit)
 constexpr uint32_t kKStages = 2, kVStages = 2;        // K and V ring depths
-constexpr uint32_t OFF_Q = 0;                         // two Q buffers (units alternate)
-constexpr uint32_t OFF_K = OFF_Q + 2 * kTileBytes;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + kQSlots * kTileBytes;
 constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
-constexpr uint32_t OFF_INVL = OFF_V + kVStages * kTileBytes;   // float[2][128]
-constexpr uint32_t OFF_BAR = OFF_INVL + 2 * 128 * 4;
+constexpr uint32_t OFF_BAR = OFF_V + kVStages * kTileBytes;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;          // + barriers + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
@@ -79,19 +88,21 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;        // 2 s per wait
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, 0, 1);
 
-// mbarrier slots (8 bytes each) at OFF_BAR
+// mbarrier slots (8 bytes each) at OFF_BAR; "X" slots come as (A, B) pairs.
 enum {
-  B_QFULL0 = 0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_SFULL0, B_SFULL1, B_PFULL0, B_PFULL1, B_PVDONE,
-  B_OFULL0, B_OFULL1,
-  B_LFULL0, B_LFULL1, B_OEMPTY0, B_OEMPTY1, B_UFULL0, B_UFULL1, B_UEMPTY0, B_UEMPTY1,
-  B_KFULL0, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
+  B_QFULL0 = 0, B_QEMPTY0 = B_QFULL0 + 3,
+  B_SFULL0 = B_QEMPTY0 + 3, B_PFULL0 = B_SFULL0 + 2, B_OFULL0 = B_PFULL0 + 2,
+  B_OEMPTY0 = B_OFULL0 + 2,
+  B_UFULL0 = B_OEMPTY0 + 2, B_UEMPTY0 = B_UFULL0 + 4,
+  B_KFULL0 = B_UEMPTY0 + 4, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
   B_COUNT = B_VEMPTY0 + 4
 };
-static_assert(kKStages <= 4 && kVStages <= 4, "ring depth");
+static_assert(kQSlots == 3 && kKStages <= 4 && kVStages <= 4, "ring depth");
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
-constexpr uint32_t OFF_UNIT = OFF_ABORT + 4;                     // int[2]
-static_assert(OFF_UNIT + 8 <= OFF_BAR + 512, "barrier area");
+constexpr uint32_t kUnitSlots = 4;                                // unit record ring depth
+constexpr uint32_t OFF_UNIT = (OFF_ABORT + 4 + 15) / 16 * 16;    // int4[kUnitSlots] unit records
+static_assert(OFF_UNIT + 16 * kUnitSlots <= OFF_BAR + 512, "barrier area");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // Position in a ring of `n` stages: stage index and mbarrier phase parity.
@@ -103,30 +114,19 @@ struct Ring {
 };
 
 struct PrefillParams {
-  uint32_t* hdr;                 // [0] error word, [1] unit counter
-  const int4* units;             // (b, h, m, lo), longest first
+  uint32_t* hdr;                 // [0] error word
+  const int32_t* cta_off;        // units of CTA c: units[cta_off[c] .. cta_off[c+1])
+  const int4* units;             // (b, h, m, loA), grouped by CTA, longest first within a CTA
   void* o;
-  int32_t n_units, N, Hq, Hkv, G;
+  int32_t N, Hq, Hkv, G;
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
 };
 
-// K-major operand (Q or K) of one 16-wide K step kk (0..7): the 128-wide
-// K extent is stored as two 64-column swizzled halves of 16 KB.
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
-  return smem_desc_sw128(base + (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u, 16u,
-                         1024u);
-}
-// MN-major V operand of K step kk (keys 16kk..16kk+15): 8-key groups are
-// 1024 B apart (SBO), the two 64-wide head-dim halves 16 KB apart (LBO).
-__device__ __forceinline__ uint64_t desc_v(uint32_t base, int kk) {
-  return smem_desc_sw128(base + (uint32_t)kk * 2048u, kHalfBytes, 1024u);
-}
-
 struct Ctx {
   uint32_t bar0;                       // address of barrier 0
   volatile int* abort;
-  volatile int* ring;                  // published unit indices, 2 slots
+  volatile int4* ring;                 // published unit records, kUnitSlots slots (x < 0: no more units)
   uint32_t* hdr;
   __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
   // Bounded wait that also gives up when another role has already failed.
@@ -151,76 +151,124 @@ struct Ctx {
     const bool ok = wait(i, parity);
     return !__any_sync(0xffffffffu, !ok);
   }
-  // Next unit index from the ring.  Single-thread roles (warp_wide = false)
+  // One arrival per warp: every lane's prior accesses are ordered before
+  // lane 0's arrive by __syncwarp.
+  __device__ void arrive_warp(int i) const {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar(i));
+  }
+  // Next unit record from the ring.  Single-thread roles (warp_wide = false)
   // release the slot themselves; warp-wide roles release it from lane 0 after
   // every lane has read it.
-  __device__ bool next_unit(uint32_t i, int lane, bool warp_wide, int* u) const {
+  __device__ bool next_unit(uint32_t i, int lane, bool warp_wide, int4* u) const {
+    const uint32_t slot = i % kUnitSlots, par = (i / kUnitSlots) & 1;
     if (warp_wide) {
-      if (!wait_warp(B_UFULL0 + (i & 1), (i >> 1) & 1)) return false;
-      *u = ring[i & 1];
+      if (!wait_warp(B_UFULL0 + slot, par)) return false;
+      *u = const_cast<const int4&>(ring[slot]);
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_UEMPTY0 + (i & 1)));
+      if (lane == 0) mbar_arrive(bar(B_UEMPTY0 + slot));
     } else {
-      if (!wait(B_UFULL0 + (i & 1), (i >> 1) & 1)) return false;
-      *u = ring[i & 1];
-      mbar_arrive(bar(B_UEMPTY0 + (i & 1)));
+      if (!wait(B_UFULL0 + slot, par)) return false;
+      *u = const_cast<const int4&>(ring[slot]);
+      mbar_arrive(bar(B_UEMPTY0 + slot));
     }
     return true;
   }
 };
 
+__device__ __forceinline__ int first_key_tile(int t, int S) {
+  const long long f = (long long)t * 128 - S + 1;
+  return f > 0 ? (int)(f / 128) : 0;
+}
+
+// The unit's two query tiles: X = 0 (A, tile m) and X = 1 (B, tile m + 1).
 struct UnitInfo {
-  int S, zq, zk, m, lo;
+  int S, zq, zk;
+  int m[2], lo[2];
+  bool hasB;
+  int L, R;                            // shared key-tile range
+  __device__ bool in(int X, int j) const { return (X == 0 || hasB) && j >= lo[X] && j <= m[X]; }
 };
 
-__device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, int u) {
+__device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const int4 U) {
   UnitInfo x;
-  const int4 U = p.units[u];
   x.S = p.span[U.y];
   x.zq = U.x * p.Hq + U.y;
   x.zk = U.x * p.Hkv + U.y / p.G;
-  x.m = U.z;
-  x.lo = U.w;
+  x.m[0] = U.z;
+  x.lo[0] = U.w;
+  x.m[1] = U.z + 1;
+  x.hasB = (long long)x.m[1] * 128 < (long long)p.N;
+  x.lo[1] = first_key_tile(x.m[1], x.S);
+  x.L = x.lo[0];
+  x.R = x.hasB ? x.m[1] : x.m[0];
   return x;
 }
 
 // ---------------------------------------------------------------------------
-// Softmax role: 128 threads own the 128 rows of the unit's query tile.
+// Softmax role: 128 threads own the 128 rows of query tile X of each unit.
 //
-// Exponentials are taken against the running maximum m of the row (log2
-// domain) without first reducing the tile: a tile whose largest score exceeds
-// m by more than 15 makes the tile's sum of 2^(s - m) reach 2^15, and only
-// then (rarely after the first tile) is the tile's exact maximum computed, m
-// raised, the row sum and O rescaled, and the tile redone.  Every exponential
-// is therefore at most 2^15, far inside fp32 and bf16 range, and O / l is
-// exact whichever m was used.  A row with no maximum yet (first tile with
-// in-window keys) takes the exact maximum directly.
+// Each S tile is handled in two halves of 64 keys.  Exponentials are taken
+// against a per-row reference m (log2 domain) without reducing the half
+// first: the row's first half with in-window keys uses m = 0, later halves
+// the current m.  Only when a half's sum of 2^(s - m) leaves [2^-15, 2^15)
+// (a score more than 15 above m, or, for the first reference, every score far
+// below 0) is the half's exact maximum taken, m moved there, the row sum, O
+// and the first half's P rescaled, and the half redone.  Every exponential
+// thus stays within 2^15 and the sum never underflows, and O / l does not
+// depend on which m was used.  P of the whole tile is written over S only
+// after both halves are done.
 // ---------------------------------------------------------------------------
-constexpr float kTileSumLimit = 32768.f;             // 2^15
+constexpr float kSumHi = 32768.f;                    // 2^15
+constexpr float kSumLo = 1.f / 32768.f;              // 2^-15
 
-// Row maximum of 128 scores, 8 independent chains.
-__device__ __forceinline__ float row_max128(const float* s) {
+// 64 scores of half hh (columns 64hh .. 64hh+63) from tensor memory, masked.
+__device__ __forceinline__ void load_half(uint32_t tS, int hh, int hi_c, int lo_c, bool edge, float* s) {
+  uint32_t sr[64];
+  tmem_ld64(tS + 64u * (uint32_t)hh, sr);
+#pragma unroll
+  for (int cc = 0; cc < 64; ++cc) s[cc] = __uint_as_float(sr[cc]);
+  if (edge) {
+#pragma unroll
+    for (int cc = 0; cc < 64; ++cc) {
+      const int col = 64 * hh + cc;
+      if (col > hi_c || col <= lo_c) s[cc] = -INFINITY;
+    }
+  }
+}
+
+__device__ __forceinline__ float max64(const float* s) {
   float mx[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) mx[k] = fmaxf(s[2 * k], s[2 * k + 1]);
 #pragma unroll
-  for (int cc = 16; cc < 128; cc += 16)
+  for (int cc = 16; cc < 64; cc += 16)
 #pragma unroll
     for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], s[cc + 2 * k], s[cc + 2 * k + 1]);
   return max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
-// p = 2^(s * c - m) for 128 scores as bf16 pairs w[64] (MUFU ex2); returns
-// the fp32 sum.
-__device__ __forceinline__ float exp_tile(const float* s, float c, float neg, uint32_t* w) {
+// Pairs of exponentials taken by the cubic on the FMA pipe (exp2_poly2) rather
+// than by MUFU ex2: one in kPolyEvery.  MUFU issues 16 ex2 per clock per SM,
+// which equals the tensor core's pace at d = 128, so moving part of the work
+// to the FMA pipe shortens the softmax, the critical path between two MMAs.
+constexpr int kPolyEvery = 8;
+
+// p = 2^(s * c - m) for 64 scores as bf16 pairs w[32]; returns the fp32 sum.
+__device__ __forceinline__ float exp_half(const float* s, float c, float neg, uint32_t* w) {
   const uint64_t c2 = f2_pack(c, c), n2 = f2_pack(neg, neg);
   uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int j = 0; j < 64; ++j) {
+  for (int j = 0; j < 32; ++j) {
     const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, n2);
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    const uint64_t p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    uint64_t p2;
+    if (j % kPolyEvery == kPolyEvery - 1) {
+      p2 = exp2_poly2(x2);
+    } else {
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+    }
     acc[j & 3] = f2_add(acc[j & 3], p2);
     float p0, p1;
     f2_unpack(p2, p0, p1);
@@ -232,194 +280,281 @@ __device__ __forceinline__ float exp_tile(const float* s, float c, float neg, ui
   return a + b;
 }
 
-__device__ __forceinline__ void mask_tile(float* s, int hi_c, int lo_c) {
-  if (hi_c < 127 || lo_c >= 0) {
-#pragma unroll
-    for (int cc = 0; cc < 128; ++cc)
-      if (cc > hi_c || cc <= lo_c) s[cc] = -INFINITY;
-  }
-}
-
 __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
-                                             float* inv_l, int warp, int lane) {
+                                             int X, int warp, int lane) {
   const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
   const int r = quarter * 32 + lane;                 // row within the query tile
   const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+  const uint32_t tS = tmem + lane_base + kColS + 128u * (uint32_t)X;
+  const uint32_t tO = tmem + lane_base + kColO + 128u * (uint32_t)X;
   const float sc = p.scale_log2;
   uint32_t tcount = 0, uc = 0;
   for (uint32_t i = 0;; ++i) {
-    int u;
-    if (!c.next_unit(i, lane, true, &u)) return;
-    if (u >= p.n_units) return;
-    const UnitInfo x = decode_unit(p, u);
-    const uint32_t tO = tmem + lane_base + kColO + 128u * (uc & 1);
-    const int i_row = x.m * 128 + r;
-    float m_run = -INFINITY, l_run = 0.f;
-    for (int kt = x.lo; kt <= x.m; ++kt, ++tcount) {
-      const uint32_t sb = tcount & 1;
-      const uint32_t tS = tmem + lane_base + kColS + 128u * sb;
-      if (!c.wait_warp(B_SFULL0 + sb, (tcount >> 1) & 1)) return;
+    int4 U;
+    if (!c.next_unit(i, lane, true, &U)) return;
+    if (U.x < 0) return;
+    const UnitInfo x = decode_unit(p, U);
+    if (X == 1 && !x.hasB) continue;
+    const int i_row = x.m[X] * 128 + r;
+    float m_run = -INFINITY, l_run = 0.f;            // m_run = -inf: no reference yet
+    for (int kt = x.lo[X]; kt <= x.m[X]; ++kt, ++tcount) {
+      if (!c.wait_warp(B_SFULL0 + X, tcount & 1)) return;
       tc_fence_after();
       const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
       const int lo_c = i_row - x.S - kt * 128;       // keys c >  lo_c are inside the window
-      float s[128];
-      {
-        uint32_t sr[128];
-        tmem_ld128(tS, sr);
+      const bool edge = hi_c < 127 || lo_c >= 0;
+      uint32_t w[64];                                // P of the tile, bf16 pairs
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc) s[cc] = __uint_as_float(sr[cc]);
-      }
-      mask_tile(s, hi_c, lo_c);
-      // rows without a maximum yet take this tile's exact maximum
-      const bool need_max = m_run == -INFINITY;
-      if (__any_sync(0xffffffffu, need_max)) {
-        const float tmax = row_max128(s);
-        if (need_max) m_run = tmax * sc;            // stays -inf if every key is masked
-      }
-      uint32_t w[64];
-      float l_tile = exp_tile(s, sc, m_run == -INFINITY ? 0.f : -m_run, w);
-      const bool redo = !(l_tile < kTileSumLimit);
-      if (__any_sync(0xffffffffu, redo)) {
-        // Rare: a score far above the running maximum.  Take the tile's exact
-        // maximum, rescale the row, and recompute the tile.
-        const float mt = row_max128(s) * sc;
-        float alpha = 1.f;
-        if (redo) {
-          alpha = ex2_approx(m_run - mt);
-          m_run = mt;
-          l_run *= alpha;
-        }
-        if (__any_sync(0xffffffffu, redo && kt > x.lo)) {
-          // O must hold every PV up to tile kt-1: wait for that PV's completion.
-          if (!c.wait_warp(B_PVDONE, (tcount - 1) & 1)) return;
-          tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t rr[32];
-            tmem_ld32(tO + cc * 32, rr);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
-            tmem_st32(tO + cc * 32, rr);
+      for (int hh = 0; hh < 2; ++hh) {
+        float s[64];
+        load_half(tS, hh, hi_c, lo_c, edge, s);
+        const bool est = m_run != -INFINITY;
+        float l_h = exp_half(s, sc, est ? -m_run : 0.f, w + 32 * hh);
+        const bool any_key = max(lo_c + 1, 64 * hh) <= min(hi_c, 64 * hh + 63);
+        const bool bad = any_key && (!(l_h < kSumHi) || (!est && l_h < kSumLo));
+        if (__any_sync(0xffffffffu, bad)) {
+          // Rare: move the reference to this half's exact maximum.
+          const float mt = max64(s) * sc;
+          float alpha = 1.f;
+          if (bad) {
+            alpha = ex2_approx(m_run - mt);          // 0 when there was no reference
+            m_run = mt;
+            l_run *= alpha;
           }
+          if (kt > x.lo[X]) {
+            // O holds every PV up to tile kt-1 (the S-ready commit of this
+            // tile covered them).
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t rr[32];
+              tmem_ld32(tO + cc * 32, rr);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
+              tmem_st32(tO + cc * 32, rr);
+            }
+          }
+          if (hh == 1) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)             // P of the first half, still in registers
+              w[j] = pack_bf16x2(__uint_as_float(w[j] << 16) * alpha,
+                                 __uint_as_float(w[j] & 0xffff0000u) * alpha);
+          }
+          l_h = exp_half(s, sc, m_run == -INFINITY ? 0.f : -m_run, w + 32 * hh);
         }
-        l_tile = exp_tile(s, sc, m_run == -INFINITY ? 0.f : -m_run, w);
+        if (!est && any_key && !bad) m_run = 0.f;   // the first reference
+        l_run += l_h;
       }
-      l_run += l_tile;
       tmem_st32(tS, w);
       tmem_st32(tS + 32, w + 32);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(c.bar(B_PFULL0 + sb));
+      c.arrive_warp(B_PFULL0 + X);
     }
-    // Hand the row's normaliser to the epilogue warpgroup.  The slot was last
-    // used by unit uc-2: wait until the epilogue has released it (a unit of
-    // one or two key tiles can otherwise get here before that epilogue ran).
-    if (!c.wait_warp(B_OEMPTY0 + (uc & 1), ((uc >> 1) & 1) ^ 1)) return;
-    inv_l[128 * (uc & 1) + r] = l_run > 0.f ? 1.f / l_run : 0.f;
-    mbar_arrive(c.bar(B_LFULL0 + (uc & 1)));
-    ++uc;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Epilogue role: 128 threads write the unit's 128 output rows.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void epilogue_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
-                                              const float* inv_l, int warp, int lane) {
-  const int quarter = warp & 3;
-  const int r = quarter * 32 + lane;
-  const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-  uint32_t uc = 0;
-  for (uint32_t i = 0;; ++i) {
-    int u;
-    if (!c.next_unit(i, lane, true, &u)) return;
-    if (u >= p.n_units) return;
-    const UnitInfo x = decode_unit(p, u);
-    const uint32_t ob = uc & 1;
-    if (!c.wait_warp(B_OFULL0 + ob, (uc >> 1) & 1)) return;
-    if (!c.wait_warp(B_LFULL0 + ob, (uc >> 1) & 1)) return;
+    // Output rows: O / l -> bf16 (round to nearest even) -> global.  The O
+    // buffer is released as soon as it is in registers, so the next unit's
+    // PVs of this tile stream can start while the stores go out.
+    if (!c.wait_warp(B_OFULL0 + X, uc & 1)) return;
     tc_fence_after();
-    const uint32_t tO = tmem + lane_base + kColO + 128u * ob;
-    const float inv = inv_l[128 * ob + r];
-    const int i_row = x.m * 128 + r;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)x.zq * p.N + (size_t)i_row) * kD;
-    const bool store = i_row < p.N;
-#pragma unroll 1
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    uint32_t pk[64];
+#pragma unroll
     for (int cc = 0; cc < 4; ++cc) {
       uint32_t rr[32];
       tmem_ld32(tO + cc * 32, rr);
-      if (store) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(rr[8 * j + 0]) * inv, __uint_as_float(rr[8 * j + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(rr[8 * j + 2]) * inv, __uint_as_float(rr[8 * j + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(rr[8 * j + 4]) * inv, __uint_as_float(rr[8 * j + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(rr[8 * j + 6]) * inv, __uint_as_float(rr[8 * j + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + cc * 32 + j * 8) = w;
-        }
-      }
+      for (int j = 0; j < 16; ++j)
+        pk[16 * cc + j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * inv, __uint_as_float(rr[2 * j + 1]) * inv);
     }
     tc_fence_before();
-    mbar_arrive(c.bar(B_OEMPTY0 + ob));
+    c.arrive_warp(B_OEMPTY0 + X);
+    if (i_row < p.N) {
+      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                             ((size_t)x.zq * p.N + (size_t)i_row) * kD);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) orow[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
     ++uc;
   }
 }
 
 // ---------------------------------------------------------------------------
-// MMA role: one thread.
+// MMA role: one thread.  tcgen05.mma issue blocks for about the length of the
+// MMA, so the tensor core idles whenever this thread is not issuing: the code
+// between MMA groups is kept to scalar bookkeeping, descriptors are built from
+// templates by adding the tile's address, and all per-stream state is scalar.
 // ---------------------------------------------------------------------------
+// Descriptor words (128-byte swizzle, 8-row groups 1024 B apart): K-major Q
+// and K tiles (two 64-column halves 16 KB apart, K step = 32 B) and the
+// MN-major V tile (8-key groups 1024 B apart, head-dim halves 16 KB apart).
+constexpr uint32_t kDescHi = sw128_hi(1024u);
+__device__ __forceinline__ uint32_t desc_qk_lo(uint32_t saddr) { return sw128_lo(saddr, 16u); }
+__device__ __forceinline__ uint32_t desc_v_lo(uint32_t saddr) { return sw128_lo(saddr, kHalfBytes); }
+
+// S = Q K^T for one 128-row query tile and one 128-key tile (8 K-steps of 16).
+__device__ __forceinline__ void mma_qk(uint32_t tS, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = ((uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u) >> 4;
+    mma_bf16_ss_lo(tS, q_lo + off, k_lo + off, hi, IDESC_QK, kk > 0 ? 1u : 0u);
+  }
+}
+// O (+)= P V with P (bf16 pairs) in tensor memory, V MN-major in shared memory.
+__device__ __forceinline__ void mma_pv(uint32_t tO, uint32_t tP, uint32_t v_lo, uint32_t hi, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_bf16_ts_lo(tO, tP + (uint32_t)kk * 8u, v_lo + (uint32_t)kk * (2048u >> 4), hi, IDESC_PV,
+                   (!first || kk > 0) ? 1u : 0u);
+}
+
+// Q slots of a unit's two tiles (A then B), in the producer's order of loads.
+struct QSlots {
+  uint32_t sA, pA, sB, pB;
+};
+__device__ __forceinline__ QSlots take_q(const UnitInfo& x, uint32_t& nq) {
+  QSlots q;
+  q.sA = nq % kQSlots;
+  q.pA = (nq / kQSlots) & 1;
+  ++nq;
+  q.sB = 0;
+  q.pB = 0;
+  if (x.hasB) {
+    q.sB = nq % kQSlots;
+    q.pB = (nq / kQSlots) & 1;
+    ++nq;
+  }
+  return q;
+}
+
 __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
                                          uint32_t sQ0, uint32_t sK0, uint32_t sV0) {
-  Ring kr, vr;                      // K and V ring positions
-  uint32_t tc = 0, tp = 0, uc = 0;  // S tiles issued, PV tiles issued, units
-  for (uint32_t i = 0;; ++i) {
-    int u;
-    if (!c.next_unit(i, 0, false, &u)) return;
-    if (u >= p.n_units) return;
-    const UnitInfo x = decode_unit(p, u);
-    const uint32_t ob = uc & 1;
-    const uint32_t tO = tmem + kColO + 128u * ob;
-    const uint32_t sQ = sQ0 + ob * kTileBytes;
-    if (!c.wait(B_QFULL0 + ob, (uc >> 1) & 1)) return;
-    tc_fence_after();
-    // PV of the unit's tile jj (P in the S buffer that tile used).
-    auto pv = [&](bool first) -> bool {
-      if (!c.wait(B_PFULL0 + (tp & 1), (tp >> 1) & 1)) return false;
-      if (!c.wait(B_VFULL0 + vr.stage, vr.phase)) return false;
-      if (first && !c.wait(B_OEMPTY0 + ob, ((uc >> 1) & 1) ^ 1)) return false;
-      tc_fence_after();
-      const uint32_t tP = tmem + kColS + 128u * (tp & 1);
-      const uint32_t sV = sV0 + vr.stage * kTileBytes;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ts(tO, tP + (uint32_t)kk * 8u, desc_v(sV, kk), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-      mma_commit(c.bar(B_PVDONE));
-      mma_commit(c.bar(B_VEMPTY0 + vr.stage));
-      vr.next(kVStages);
-      ++tp;
-      return true;
-    };
-    for (int kt = x.lo; kt <= x.m; ++kt) {
-      // S(kt) = Q K(kt)^T into S buffer tc & 1
-      if (!c.wait(B_KFULL0 + kr.stage, kr.phase)) return;
-      tc_fence_after();
-      const uint32_t sK = sK0 + kr.stage * kTileBytes;
-      const uint32_t tS = tmem + kColS + 128u * (tc & 1);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tS, desc_kmajor(sQ, kk), desc_kmajor(sK, kk), IDESC_QK, kk > 0 ? 1u : 0u);
-      mma_commit(c.bar(B_SFULL0 + (tc & 1)));
-      mma_commit(c.bar(B_KEMPTY0 + kr.stage));
-      kr.next(kKStages);
-      ++tc;
-      if (kt == x.m) mma_commit(c.bar(B_QEMPTY0 + ob));   // every S of the unit issued
-      // O += P(kt-1) V(kt-1)
-      if (kt > x.lo && !pv(kt - 1 == x.lo)) return;
+  const uint32_t hi = kDescHi;
+  const uint32_t tSA = tmem + kColS, tSB = tmem + kColS + 128u;
+  const uint32_t tOA = tmem + kColO, tOB = tmem + kColO + 128u;
+  uint32_t kst = 0, kph = 0, vst = 0, vph = 0;       // K and V ring positions
+  uint32_t nq = 0;                                   // Q tiles used so far (slot nq % 3)
+  uint32_t tpA = 0, tpB = 0, ucA = 0, ucB = 0;       // PV tiles and units per stream
+  uint32_t ui = 0;                                   // unit records read
+  int4 U;
+  if (!c.next_unit(ui++, 0, false, &U)) return;
+  if (U.x < 0) return;
+  UnitInfo x = decode_unit(p, U);
+  QSlots q = take_q(x, nq);
+  bool started_A = false;                            // S_A(L) of x already issued
+  while (true) {
+    bool qrB = false;
+    // prologue: the S tiles of key tile L (tile A always starts at L; its S
+    // may have been issued during the previous unit's last step)
+    if (!c.wait(B_KFULL0 + kst, kph)) return;
+    {
+      const uint32_t dk = desc_qk_lo(sK0 + kst * kTileBytes);
+      if (!started_A) {
+        if (!c.wait(B_QFULL0 + q.sA, q.pA)) return;
+        tc_fence_after();
+        mma_qk(tSA, desc_qk_lo(sQ0 + q.sA * kTileBytes), dk, hi);
+        mma_commit(c.bar(B_SFULL0));
+        if (x.L == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
+      }
+      if (x.in(1, x.L)) {
+        if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
+        qrB = true;
+        tc_fence_after();
+        mma_qk(tSB, desc_qk_lo(sQ0 + q.sB * kTileBytes), dk, hi);
+        mma_commit(c.bar(B_SFULL0 + 1));
+      }
     }
-    if (!pv(x.m == x.lo)) return;                   // last tile's PV
-    mma_commit(c.bar(B_OFULL0 + ob));
-    ++uc;
+    mma_commit(c.bar(B_KEMPTY0 + kst));
+    if (++kst == kKStages) { kst = 0; kph ^= 1u; }
+    // next unit, when its tile A could start during this unit's last step
+    bool have_next = false, ended = false;
+    int4 Uy = make_int4(0, 0, 0, 0);
+    uint32_t ysA = 0, ypA = 0;
+    for (int j = x.L; j <= x.R; ++j) {
+      const bool more = j < x.R;
+      if (!c.wait(B_VFULL0 + vst, vph)) return;
+      const uint32_t dv = desc_v_lo(sV0 + vst * kTileBytes);
+      const uint32_t dk = desc_qk_lo(sK0 + kst * kTileBytes);   // K(j+1) when more
+      if (more && !c.wait(B_KFULL0 + kst, kph)) return;
+      // stream A: O_A += P_A(j) V(j), then S_A(j+1)
+      if (j <= x.m[0]) {
+        if (!c.wait(B_PFULL0, tpA & 1)) return;
+        const bool first = j == x.lo[0];
+        if (first && !c.wait(B_OEMPTY0, (ucA & 1) ^ 1)) return;
+        tc_fence_after();
+        mma_pv(tOA, tSA, dv, hi, first);
+        ++tpA;
+        if (j == x.m[0]) {
+          mma_commit(c.bar(B_OFULL0));
+          ++ucA;
+        } else {
+          mma_qk(tSA, desc_qk_lo(sQ0 + q.sA * kTileBytes), dk, hi);   // j + 1 <= m_A, so more
+          mma_commit(c.bar(B_SFULL0));               // also covers PV_A(j)
+          if (j + 1 == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
+        }
+      } else if (!more) {
+        // Last step, tile B only: S_A of the next unit's first key tile (the
+        // next K in the ring) goes to the tensor core now, so tile A's
+        // softmax starts the next unit while tile B finishes this one.
+        if (!c.next_unit(ui++, 0, false, &Uy)) return;
+        if (Uy.x < 0) {
+          ended = true;
+        } else {
+          // tile A of the next unit: query tile Uy.z, first key tile Uy.w; its
+          // Q slot is the next in the rotation
+          ysA = nq % kQSlots;
+          ypA = (nq / kQSlots) & 1;
+          if (!c.wait(B_KFULL0 + kst, kph)) return;
+          if (!c.wait(B_QFULL0 + ysA, ypA)) return;
+          tc_fence_after();
+          mma_qk(tSA, desc_qk_lo(sQ0 + ysA * kTileBytes), desc_qk_lo(sK0 + kst * kTileBytes), hi);
+          mma_commit(c.bar(B_SFULL0));
+          if (Uy.w == Uy.z) mma_commit(c.bar(B_QEMPTY0 + ysA));
+          have_next = true;
+        }
+      }
+      // stream B: O_B += P_B(j) V(j), then S_B(j+1)
+      if (x.hasB) {
+        if (j >= x.lo[1]) {
+          if (!c.wait(B_PFULL0 + 1, tpB & 1)) return;
+          const bool first = j == x.lo[1];
+          if (first && !c.wait(B_OEMPTY0 + 1, (ucB & 1) ^ 1)) return;
+          tc_fence_after();
+          mma_pv(tOB, tSB, dv, hi, first);
+          ++tpB;
+          if (j == x.m[1]) {
+            mma_commit(c.bar(B_OFULL0 + 1));
+            ++ucB;
+          }
+        }
+        if (more && j + 1 >= x.lo[1]) {
+          if (!qrB) {
+            if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
+            qrB = true;
+            tc_fence_after();
+          }
+          mma_qk(tSB, desc_qk_lo(sQ0 + q.sB * kTileBytes), dk, hi);
+          mma_commit(c.bar(B_SFULL0 + 1));
+          if (j + 1 == x.m[1]) mma_commit(c.bar(B_QEMPTY0 + q.sB));
+        }
+      }
+      mma_commit(c.bar(B_VEMPTY0 + vst));
+      if (++vst == kVStages) { vst = 0; vph ^= 1u; }
+      if (more) {
+        mma_commit(c.bar(B_KEMPTY0 + kst));
+        if (++kst == kKStages) { kst = 0; kph ^= 1u; }
+      }
+    }
+    if (ended) return;
+    if (have_next) {
+      x = decode_unit(p, Uy);
+      q = take_q(x, nq);                             // slot of tile A = ysA
+      started_A = true;
+      continue;
+    }
+    if (!c.next_unit(ui++, 0, false, &U)) return;
+    if (U.x < 0) return;
+    x = decode_unit(p, U);
+    q = take_q(x, nq);
+    started_A = false;
   }
 }
 
@@ -431,35 +566,70 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
                                               const CUtensorMap* tmV, uint32_t sQ0, uint32_t sK0,
                                               uint32_t sV0) {
   Ring kr, vr;
-  uint32_t qc = 0;
+  uint32_t nq = 0;
+  auto load_q = [&](int m, int zq) -> bool {
+    const uint32_t slot = nq % kQSlots, par = (nq / kQSlots) & 1;
+    ++nq;
+    if (!c.wait(B_QEMPTY0 + slot, par ^ 1)) return false;
+    const uint32_t sQ = sQ0 + slot * kTileBytes;
+    mbar_expect_tx(c.bar(B_QFULL0 + slot), kTileBytes);
+    tma_load_3d(sQ, tmQ, c.bar(B_QFULL0 + slot), 0, m * 128, zq);
+    tma_load_3d(sQ + kHalfBytes, tmQ, c.bar(B_QFULL0 + slot), 64, m * 128, zq);
+    return true;
+  };
+  auto load_k = [&](int kt, int zk) -> bool {
+    const uint32_t ks = kr.stage;
+    if (!c.wait(B_KEMPTY0 + ks, kr.phase ^ 1)) return false;
+    kr.next(kKStages);
+    mbar_expect_tx(c.bar(B_KFULL0 + ks), kTileBytes);
+    tma_load_3d(sK0 + ks * kTileBytes, tmK, c.bar(B_KFULL0 + ks), 0, kt * 128, zk);
+    tma_load_3d(sK0 + ks * kTileBytes + kHalfBytes, tmK, c.bar(B_KFULL0 + ks), 64, kt * 128, zk);
+    return true;
+  };
+  auto load_v = [&](int kt, int zk) -> bool {
+    const uint32_t vs = vr.stage;
+    if (!c.wait(B_VEMPTY0 + vs, vr.phase ^ 1)) return false;
+    vr.next(kVStages);
+    mbar_expect_tx(c.bar(B_VFULL0 + vs), kTileBytes);
+    tma_load_3d(sV0 + vs * kTileBytes, tmV, c.bar(B_VFULL0 + vs), 0, kt * 128, zk);
+    tma_load_3d(sV0 + vs * kTileBytes + kHalfBytes, tmV, c.bar(B_VFULL0 + vs), 64, kt * 128, zk);
+    return true;
+  };
   for (uint32_t i = 0;; ++i) {
-    if (!c.wait(B_UEMPTY0 + (i & 1), ((i >> 1) & 1) ^ 1)) return;
-    const int u = (int)atomicAdd(p.hdr + 1, 1u);
-    c.ring[i & 1] = u;
-    mbar_arrive(c.bar(B_UFULL0 + (i & 1)));
-    if (u >= p.n_units) return;
-    const UnitInfo x = decode_unit(p, u);
-    const uint32_t qb = qc & 1;
-    if (!c.wait(B_QEMPTY0 + qb, ((qc >> 1) & 1) ^ 1)) return;
-    ++qc;
-    const uint32_t sQ = sQ0 + qb * kTileBytes;
-    mbar_expect_tx(c.bar(B_QFULL0 + qb), kTileBytes);
-    tma_load_3d(sQ, tmQ, c.bar(B_QFULL0 + qb), 0, x.m * 128, x.zq);
-    tma_load_3d(sQ + kHalfBytes, tmQ, c.bar(B_QFULL0 + qb), 64, x.m * 128, x.zq);
-    for (int kt = x.lo; kt <= x.m; ++kt) {
-      const uint32_t ks = kr.stage;
-      if (!c.wait(B_KEMPTY0 + ks, kr.phase ^ 1)) return;
-      kr.next(kKStages);
-      mbar_expect_tx(c.bar(B_KFULL0 + ks), kTileBytes);
-      tma_load_3d(sK0 + ks * kTileBytes, tmK, c.bar(B_KFULL0 + ks), 0, kt * 128, x.zk);
-      tma_load_3d(sK0 + ks * kTileBytes + kHalfBytes, tmK, c.bar(B_KFULL0 + ks), 64, kt * 128, x.zk);
-      const uint32_t vs = vr.stage;
-      if (!c.wait(B_VEMPTY0 + vs, vr.phase ^ 1)) return;
-      vr.next(kVStages);
-      mbar_expect_tx(c.bar(B_VFULL0 + vs), kTileBytes);
-      tma_load_3d(sV0 + vs * kTileBytes, tmV, c.bar(B_VFULL0 + vs), 0, kt * 128, x.zk);
-      tma_load_3d(sV0 + vs * kTileBytes + kHalfBytes, tmV, c.bar(B_VFULL0 + vs), 64, kt * 128, x.zk);
+    int4 U;
+    if (!c.next_unit(i, 0, false, &U)) return;
+    if (U.x < 0) return;
+    const UnitInfo x = decode_unit(p, U);
+    // Loads in the MMA's order of use: Q_A, K(L), then per key tile j:
+    // V(j), K(j+1); Q_B right before the first K tile that tile B uses.
+    if (!load_q(x.m[0], x.zq)) return;
+    if (!load_k(x.L, x.zk)) return;
+    if (x.hasB && x.lo[1] == x.L && !load_q(x.m[1], x.zq)) return;
+    for (int j = x.L; j <= x.R; ++j) {
+      if (!load_v(j, x.zk)) return;
+      if (j < x.R) {
+        if (x.hasB && x.lo[1] == j + 1 && !load_q(x.m[1], x.zq)) return;
+        if (!load_k(j + 1, x.zk)) return;
+      }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Unit fetcher: one thread publishes the records of this CTA's units (a
+// balanced list built on the host) up to kUnitSlots ahead of the slowest
+// consumer, then a record with x < 0; no role waits on a global load.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fetcher_role(const PrefillParams& p, const Ctx& c) {
+  const int first = p.cta_off[blockIdx.x], last = p.cta_off[blockIdx.x + 1];
+  for (uint32_t i = 0;; ++i) {
+    const uint32_t slot = i % kUnitSlots;
+    if (!c.wait(B_UEMPTY0 + slot, ((i / kUnitSlots) & 1) ^ 1)) return;
+    const int u = first + (int)i;
+    const int4 U = u < last ? p.units[u] : make_int4(-1, 0, 0, 0);
+    const_cast<int4&>(c.ring[slot]) = U;
+    mbar_arrive(c.bar(B_UFULL0 + slot));
+    if (U.x < 0) return;
   }
 }
 
@@ -477,18 +647,16 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   Ctx c;
   c.bar0 = sbase + OFF_BAR;
   c.abort = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
-  c.ring = reinterpret_cast<volatile int*>(smem + OFF_UNIT);
+  c.ring = reinterpret_cast<volatile int4*>(smem + OFF_UNIT);
   c.hdr = p.hdr;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
-  float* inv_l = reinterpret_cast<float*>(smem + OFF_INVL);
 
   if (tid == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PFULL0 || i == B_PFULL1 || i == B_LFULL0 || i == B_LFULL1 || i == B_OEMPTY0 ||
-          i == B_OEMPTY1)
-        cnt = 128;
-      if (i == B_UEMPTY0 || i == B_UEMPTY1) cnt = 9;   // MMA thread + 4 softmax + 4 epilogue warps
+      if ((i >= B_PFULL0 && i < B_PFULL0 + 2) || (i >= B_OEMPTY0 && i < B_OEMPTY0 + 2))
+        cnt = 4;                                        // one arrival per warp of a warpgroup
+      if (i >= B_UEMPTY0 && i < B_UEMPTY0 + (int)kUnitSlots) cnt = 10;   // producer, MMA, 2 x 4 softmax warps
       mbar_init(c.bar(i), cnt);
     }
     *c.abort = 0;
@@ -504,17 +672,16 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    regs_dec<kRegsControl>();
+    if constexpr (kRegsControl < kRegsLaunch) regs_dec<kRegsControl>();
     if (warp == 0 && lane == 0)
       producer_role(p, c, &tmQ, &tmK, &tmV, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
+    else if (warp == 2 && lane == 0)
+      fetcher_role(p, c);
     else if (warp == 1 && lane == 0)
       mma_role(p, c, tmem, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
-  } else if (warp < 8) {
-    regs_inc<kRegsSoftmax>();
-    softmax_role(p, c, tmem, inv_l, warp, lane);
   } else {
-    regs_dec<kRegsEpilogue>();
-    epilogue_role(p, c, tmem, inv_l, warp, lane);
+    regs_inc<kRegsSoftmax>();
+    softmax_role(p, c, tmem, warp < 8 ? 0 : 1, warp, lane);
   }
 
   // teardown: after a timeout give in-flight copies and MMAs time to land
@@ -558,7 +725,9 @@ bool make_map(CUtensorMap* map, const void* ptr, int32_t N, int64_t heads) {
   return r == CUDA_SUCCESS;
 }
 
-constexpr size_t kUnitsOffset = 256;
+constexpr size_t kOffsOffset = 256;                          // int32 cta_off[kMaxCtas + 1]
+constexpr size_t kUnitsOffset = kOffsOffset + (4 * (kPrefillMaxCtas + 1) + 15) / 16 * 16;
+constexpr int64_t kUnitOverheadTiles = 4;     // per-unit pipeline fill/drain, in tile steps
 
 int64_t first_tile_host(int64_t qt, int32_t S) {
   return std::max<int64_t>(0, qt * kTileM - S + 1) / kTileN;
@@ -566,27 +735,69 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 
 }  // namespace
 
-// Units of one 128-row query tile; a unit's cost is its number of key tiles.
-std::vector<int32_t> prefill_units(int32_t B, int32_t Hq, int32_t N, const int32_t* spans) {
+// Units of two consecutive 128-row query tiles (m, m + 1) of one head, sorted
+// longest first and dealt to n_ctas lists by the greedy longest-processing-
+// time rule (each unit to the list with the least work so far); a unit's work
+// is its (query tile, key tile) pairs plus a fixed per-unit overhead.
+PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas) {
   const int64_t M = (N + kTileM - 1) / kTileM;      // query tiles
   struct U { int32_t b, h, m, lo; int64_t cost; };
   std::vector<U> v;
-  v.reserve((size_t)B * Hq * M);
+  v.reserve((size_t)B * Hq * ((M + 1) / 2));
   for (int32_t b = 0; b < B; ++b)
     for (int32_t h = 0; h < Hq; ++h)
-      for (int64_t m = 0; m < M; ++m) {
+      for (int64_t m = 0; m < M; m += 2) {
         const int64_t lo = first_tile_host(m, spans[h]);
-        v.push_back({b, h, (int32_t)m, (int32_t)lo, m - lo + 1});
+        int64_t cost = m - lo + 1 + kUnitOverheadTiles;
+        if (m + 1 < M) cost += m + 1 - first_tile_host(m + 1, spans[h]) + 1;
+        v.push_back({b, h, (int32_t)m, (int32_t)lo, cost});
       }
   std::stable_sort(v.begin(), v.end(), [](const U& a, const U& c) { return a.cost > c.cost; });
-  std::vector<int32_t> out(v.size() * 4);
+  const int32_t n = (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_ctas, (int64_t)v.size()));
+  std::vector<std::vector<int32_t>> lists(n);
+  using Slot = std::pair<int64_t, int32_t>;          // (work so far, list)
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int32_t c = 0; c < n; ++c) heap.push({0, c});
   for (size_t i = 0; i < v.size(); ++i) {
-    out[4 * i + 0] = v[i].b;
-    out[4 * i + 1] = v[i].h;
-    out[4 * i + 2] = v[i].m;
-    out[4 * i + 3] = v[i].lo;
+    Slot sl = heap.top();
+    heap.pop();
+    lists[sl.second].push_back((int32_t)i);
+    sl.first += v[i].cost;
+    heap.push(sl);
+  }
+  PrefillSchedule out;
+  out.n_ctas = n;
+  out.off.assign(n + 1, 0);
+  out.units.reserve(v.size() * 4);
+  for (int32_t c = 0; c < n; ++c) {
+    for (int32_t i : lists[c]) {
+      out.units.push_back(v[i].b);
+      out.units.push_back(v[i].h);
+      out.units.push_back(v[i].m);
+      out.units.push_back(v[i].lo);
+    }
+    out.off[c + 1] = (int32_t)(out.units.size() / 4);
   }
   return out;
+}
+
+// One row (CTA, unit, b, h, query tile, first key tile, last key tile) per
+// query tile, in the order each CTA takes its units.
+std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, const int32_t* spans,
+                                           int32_t n_ctas) {
+  const int64_t M = (N + kTileM - 1) / kTileM;
+  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, n_ctas);
+  std::vector<int32_t> rows;
+  rows.reserve((size_t)B * Hq * M * 7);
+  for (int32_t c = 0; c < sch.n_ctas; ++c)
+    for (int32_t i = sch.off[c]; i < sch.off[c + 1]; ++i) {
+      const int32_t b = sch.units[4 * i], h = sch.units[4 * i + 1], m = sch.units[4 * i + 2];
+      for (int32_t t = m; t <= m + 1 && t < M; ++t) {
+        const int32_t row[7] = {c, i, b, h, t, (int32_t)first_tile_host(t, spans[h]), t};
+        rows.insert(rows.end(), row, row + 7);
+      }
+    }
+  return rows;
 }
 
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
@@ -603,21 +814,24 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
   if (!make_map(&mq, q, N, (int64_t)B * Hq) || !make_map(&mk, k, N, (int64_t)B * Hkv) ||
       !make_map(&mv, v, N, (int64_t)B * Hkv))
     return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
-  // Header (error word, unit counter, zeroed) and the longest-first unit list,
+  // Header (error word, zeroed), the per-CTA list offsets and the units,
   // uploaded in one copy.  The pageable source is staged by the runtime
   // before cudaMemcpyAsync returns.
-  std::vector<int32_t> units = prefill_units(B, Hq, N, spans);
-  const size_t n_units = units.size() / 4;
-  std::vector<int32_t> blob(kUnitsOffset / 4 + units.size(), 0);
-  std::copy(units.begin(), units.end(), blob.begin() + kUnitsOffset / 4);
+  const int64_t M = (N + kTileM - 1) / kTileM;
+  const int64_t n_units = (int64_t)B * Hq * ((M + 1) / 2);
+  const int32_t grid = (int32_t)std::min<int64_t>({n_units, (int64_t)sm_count(), (int64_t)kPrefillMaxCtas});
+  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, grid);
+  std::vector<int32_t> blob(kUnitsOffset / 4 + sch.units.size(), 0);
+  std::copy(sch.off.begin(), sch.off.end(), blob.begin() + kOffsOffset / 4);
+  std::copy(sch.units.begin(), sch.units.end(), blob.begin() + kUnitsOffset / 4);
   cudaError_t e = cudaMemcpyAsync(ws, blob.data(), blob.size() * 4, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefill unit upload");
 
   PrefillParams p;
   p.hdr = reinterpret_cast<uint32_t*>(ws);
+  p.cta_off = reinterpret_cast<const int32_t*>((char*)ws + kOffsOffset);
   p.units = reinterpret_cast<const int4*>((char*)ws + kUnitsOffset);
   p.o = o;
-  p.n_units = (int32_t)n_units;
   p.N = N;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -632,8 +846,7 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "prefill smem attribute");
-  const int grid = (int)std::min<size_t>(n_units, (size_t)sm_count());
-  prefill_bf16_sm100_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, p);
+  prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, p);
   return check_launch("prefill_bf16 launch");
 }
 

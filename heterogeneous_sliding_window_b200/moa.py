@@ -63,7 +63,7 @@ def load():
         "moa_workspace_check": (ctypes.c_int, [vp, vp]),
         "moa_prefill": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_int, P(i32), f32,
                                        vp, sz, vp, vp]),
-        "moa_prefill_schedule": (ctypes.c_int, [i32, i32, i64, P(i32), P(i32), i64, P(i64)]),
+        "moa_prefill_schedule": (ctypes.c_int, [i32, i32, i64, P(i32), i32, P(i32), i64, P(i64)]),
         "moa_decode": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_static_ws": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp]),
     }
@@ -204,13 +204,15 @@ def moa_prefill(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, scale, ws=None, ws_b
                               float(scale), _ptr(ws), ws_bytes, fill, _stream(stream)), "moa_prefill")
 
 
-def moa_prefill_schedule(B, Hq, N, spans):
+def moa_prefill_schedule(B, Hq, N, spans, n_ctas):
     sp, spp = _i32(spans)
     n = ctypes.c_int64()
-    _check(load().moa_prefill_schedule(B, Hq, int(N), spp, None, 0, ctypes.byref(n)), "moa_prefill_schedule")
-    out = np.zeros((n.value, 6), dtype=np.int32)
-    _check(load().moa_prefill_schedule(B, Hq, int(N), spp, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-                                       n.value, ctypes.byref(n)), "moa_prefill_schedule")
+    _check(load().moa_prefill_schedule(B, Hq, int(N), spp, int(n_ctas), None, 0, ctypes.byref(n)),
+           "moa_prefill_schedule")
+    out = np.zeros((n.value, 7), dtype=np.int32)
+    _check(load().moa_prefill_schedule(B, Hq, int(N), spp, int(n_ctas),
+                                       out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n.value,
+                                       ctypes.byref(n)), "moa_prefill_schedule")
     return out
 
 

@@ -168,14 +168,20 @@ moa_status moa_prefill(const void* q, const void* k, const void* v, void* o,
                        void* workspace, size_t ws_bytes, moa_kv_cache* fill_or_null,
                        void* stream);
 
-/* Host view of the prefill schedule.  The kernel's work unit is one query
- * tile of 128 rows of one (sequence, head); units run longest first.  One row
- * of 6 int32 per unit, in the order the persistent kernel takes them:
- * (unit, b, h, m, lo, hi) -- query rows [128m, 128m+127] visit key tiles
+/* Host view of the prefill schedule.  The kernel's work unit is two
+ * consecutive query tiles of 128 rows (m, m+1) of one (sequence, head),
+ * sharing one stream of key/value tiles (a head with an odd number of query
+ * tiles ends with a one-tile unit).  Units are sorted longest first and dealt
+ * to n_ctas per-CTA lists (1 <= n_ctas <= 1024; moa_prefill uses the number
+ * of SMs, or fewer when there are fewer units) by the greedy
+ * longest-processing-time rule.  One row of 7 int32 per query tile, a unit's
+ * rows adjacent, each CTA's units in the order it runs them:
+ * (cta, unit, b, h, m, lo, hi) -- query rows [128m, 128m+127] visit key tiles
  * lo..hi of 128 keys (hi = m, the diagonal tile).  Writes min(cap, n) rows,
  * *n_rows_out = n.  Host only. */
 moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
-                                int32_t* rows_out, int64_t cap, int64_t* n_rows_out);
+                                int32_t n_ctas, int32_t* rows_out, int64_t cap,
+                                int64_t* n_rows_out);
 
 /* ---------------------------------------------------------------------------
  * Decode: one new query token per sequence against the ring cache.  Call

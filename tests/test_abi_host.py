@@ -91,30 +91,55 @@ def _tiles_needed_brute(m, S, N):
     return need
 
 
-@pytest.mark.parametrize("N,spans", [(1000, [1, 64, 127, 128, 129, 300, 1000, 5000]), (128, [1, 128]),
-                                     (129, [2, 129]), (5, [3]), (640, [256, 700])])
-def test_prefill_schedule_covers_band(N, spans):
+@pytest.mark.parametrize("N,spans,n_ctas", [(1000, [1, 64, 127, 128, 129, 300, 1000, 5000], 7),
+                                            (128, [1, 128], 148), (129, [2, 129], 3), (5, [3], 1),
+                                            (640, [256, 700], 2), (8192, [64, 4736, 576, 5568], 148)])
+def test_prefill_schedule_covers_band(N, spans, n_ctas):
     B = 2
     Hq = len(spans)
-    rows = moa.moa_prefill_schedule(B, Hq, N, spans)
+    rows = moa.moa_prefill_schedule(B, Hq, N, spans, n_ctas)
     M = (N + 127) // 128
-    assert rows.shape == (B * Hq * M, 6)
+    assert rows.shape == (B * Hq * M, 7)
     seen = set()
-    unit_cost = {}
+    unit_tiles = {}
+    unit_cta = {}
     order = []
-    for unit, b, h, m, lo, hi in rows.tolist():
+    for cta, unit, b, h, m, lo, hi in rows.tolist():
         assert (b, h, m) not in seen
         seen.add((b, h, m))
         assert hi == m
-        need = _tiles_needed_brute(m, spans[h], N)
+        need = _tiles_needed_brute(m, spans[h], N) if N <= 1000 else set(
+            range(max(0, 128 * m - spans[h] + 1) // 128, m + 1))
         assert set(range(lo, hi + 1)) == need   # exactly the band's tiles, none skipped, none extra
-        unit_cost[unit] = unit_cost.get(unit, 0) + hi - lo + 1
+        unit_tiles.setdefault(unit, []).append((m, lo, hi))
+        assert unit_cta.setdefault(unit, cta) == cta
         if not order or order[-1] != unit:
             order.append(unit)
     assert len(seen) == B * Hq * M
-    assert order == sorted(order)               # rows of a unit are adjacent
-    costs = [unit_cost[u] for u in order]
-    assert costs == sorted(costs, reverse=True)  # longest first
+    assert order == sorted(order)               # rows of a unit adjacent, units numbered in run order
+    n_used = len(set(unit_cta.values()))
+    assert n_used == min(n_ctas, len(order))
+    # a unit is two consecutive query tiles of one head (one tile only at a head's end)
+    for unit, ts in unit_tiles.items():
+        ms = [t[0] for t in ts]
+        assert ms[0] % 2 == 0 and ms == list(range(ms[0], ms[0] + len(ms))) and len(ms) <= 2
+    # each CTA runs its units longest first; the lists are balanced within one unit (greedy LPT bound)
+    cost = {u: sum(hi - lo + 1 for _, lo, hi in ts) + 4 for u, ts in unit_tiles.items()}
+    load = {}
+    for u in order:
+        c = unit_cta[u]
+        load.setdefault(c, []).append(cost[u])
+    for c, cs in load.items():
+        assert cs == sorted(cs, reverse=True)
+    totals = [sum(cs) for cs in load.values()]
+    assert max(totals) - min(totals) <= max(cost.values())
+
+
+def test_prefill_schedule_arguments():
+    with pytest.raises(moa.MoaError):
+        moa.moa_prefill_schedule(1, 1, 128, [64], 0)
+    with pytest.raises(moa.MoaError):
+        moa.moa_prefill_schedule(1, 1, 128, [64], 1025)
 
 
 def test_kv_sizes_match_layout():

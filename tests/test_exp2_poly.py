@@ -1,4 +1,4 @@
-"""Error bound of the FMA-pipe 2^x the prefill kernel uses for a quarter of its exponentials.
+"""Error bound of the FMA-pipe 2^x the prefill kernel uses for one pair of exponentials in eight.
 
 The kernel's exp2_poly (csrc/sm100.cuh) reduces x = n + f, n = round(x), evaluates
 a fitted cubic for 2^f and adds n into the exponent field.  This test replays
