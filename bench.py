@@ -355,6 +355,7 @@ def run_ours(args):
     e2e_ms = e2e_ms.item()
     h2d = sum(x.numel() * x.element_size() for x in h_q + h_k + h_v)
     d2h = sum(x.numel() * x.element_size() for x in h_o)
+    gqa = gqa_decode_layer(stream)
 
     result = None
     if rank == 0:
@@ -387,6 +388,7 @@ def run_ours(args):
             "e2e": {"value": round(ws_n * D_B / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "note": "decode step through the C ABI from pinned host q/k/v to host o"},
+            "gqa_decode": gqa,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clock_info,
             "cpu_baseline": {"value": round(cpu_tok, 4), "unit": "tokens/s", "cores": _oracle_threads(),
@@ -397,6 +399,51 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def gqa_decode_layer(stream, reps=20):
+    """One Llama3-8B-shaped grouped-query decode layer (B=32, 32 query heads on 8 KV heads,
+    d=128, context 8192, per-head spans at 50% density), timed back to back with CUDA events.
+
+    Bytes are those of the group-shared read: every cached row of each group's longest window
+    once, plus q and o.
+    """
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    B, Hq, Hkv, D, N = 32, 32, 8, 128, 8192
+    a, b = inputs.tables_7b(1001, Hq, N, BLOCK, 0.5, moa.moa_rules_eval)
+    sp = moa.moa_rules_eval(a, b, N, BLOCK)
+    G = Hq // Hkv
+    caps = [max(sp[g * G:(g + 1) * G]) for g in range(Hkv)]
+    c = moa.KVCache(B, Hkv, D, "bf16", caps)
+    data = c.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(2000, (data.numel(),)))
+    c.set_positions([N] * B)
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, D, sp)
+    q = inputs.randn_cuda(2001, (B, Hq, D))
+    o = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(D)
+    for _ in range(3):
+        moa.moa_decode(c.handle, q, o, Hq, sp, scale, ws.ptr, ws.nbytes, stream)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        moa.moa_decode(c.handle, q, o, Hq, sp, scale, ws.ptr, ws.nbytes, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    c.positions()
+    ms = e0.elapsed_time(e1) / reps
+    group_bytes = B * sum(2 * cp * D * 2 for cp in caps) + 2 * B * Hq * D * 2
+    head_bytes = B * sum(2 * S * D * 2 for S in sp) + 2 * B * Hq * D * 2
+    group_path = sum(sp) * 10 > sum(caps) * 22
+    c.close()
+    return {"workload": "llama3-8b-shaped decode layer: B=%d Hq=%d Hkv=%d d=%d ctx %d density 0.50" % (B, Hq, Hkv, D, N),
+            "kernel": "decode_group_kernel<bf16,128,4>" if group_path else "decode_kernel<bf16,128>",
+            "ms": round(ms, 4), "group_window_bytes": group_bytes, "per_head_window_bytes": head_bytes,
+            "gbs_of_group_bytes": round(group_bytes / (ms * 1e-3) / 1e9, 1),
+            "tokens_per_s_one_layer": round(B / (ms * 1e-3), 1)}
 
 
 def _ncu_traffic():

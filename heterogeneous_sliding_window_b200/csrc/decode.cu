@@ -43,7 +43,8 @@ struct DecodeParams {
   float scale_log2;
   int64_t sumC;
   int32_t span[MOA_MAX_HEADS];
-  int32_t split_pre[MOA_MAX_HEADS + 1];
+  int32_t split_pre[MOA_MAX_HEADS + 1];   // per query head (per KV group in the group kernel)
+  int32_t hslot_pre[MOA_MAX_HEADS + 1];   // group kernel: first partial slot of each query head
   int32_t cap[MOA_MAX_HEADS];
   int64_t goff[MOA_MAX_HEADS];
 };
@@ -237,6 +238,229 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode for grouped-query attention with the K/V reads shared by the group.
+//
+// The G query heads of KV group g read windows that all end at the newest
+// position and differ only in length, so every cached row of the group's
+// longest window is loaded once and applied to each head whose window covers
+// it.  Grid: one CTA per (sequence b, group g, split s of the group's window
+// of W = min(t_b, C_g) entries); the row groups and batches are those of
+// decode_kernel, with G online softmaxes per row group instead of one.  The
+// last split of (b, g) to finish merges the partials of all G heads.  Bytes
+// read per step drop from the sum of the heads' windows to the group's
+// longest window.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int VE = Vec16<T>::N;
+  constexpr int LPR = D / VE;
+  constexpr int RPW = 32 / LPR;
+  constexpr int NG = RPW * kDecWarps;
+  constexpr int U = G >= 8 ? 4 : 6;   // rows per batch (registers: G q and accumulator vectors)
+  static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row must map onto a warp");
+
+  __shared__ float g_acc[NG][D];
+  __shared__ float g_m[NG], g_l[NG];
+  __shared__ int last_flag;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int grp = warp * RPW + sub;
+
+  const int item = blockIdx.x;
+  const int b = item / p.items_per_b;
+  const int r = item - b * p.items_per_b;
+  const int Hkv = p.Hq / G;
+  int lo = 0, hi = Hkv - 1;           // group g: last g with split_pre[g] <= r
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.split_pre[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  const int g = lo;
+  const int s = r - p.split_pre[g];
+  const int nsplit = p.split_pre[g + 1] - p.split_pre[g];
+  const int C = p.cap[g];
+  const int64_t tb = p.t[b];
+  const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);   // the group's longest window
+  const int w0 = s * kChunk;
+  const int nrows = max(0, min(kChunk, W - w0));
+  const int64_t pos0 = tb - W + w0;
+  const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
+
+  const T* Kb = reinterpret_cast<const T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
+  const T* Vb = Kb + (size_t)C * D;
+
+  // head j of the group sees window entries e >= e0[j] (e counts from the
+  // oldest entry of the group's window)
+  float qf[G][VE];
+  int e0[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const int h = g * G + j;
+    const int Sh = (int)(tb < (int64_t)p.span[h] ? tb : (int64_t)p.span[h]);
+    e0[j] = W - Sh;
+    const int4 raw = __ldg(reinterpret_cast<const int4*>(
+        reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D + li * VE));
+    Vec16<T>::cvt(raw, qf[j]);
+#pragma unroll
+    for (int e = 0; e < VE; ++e) qf[j][e] *= p.scale_log2;
+  }
+
+  float m[G], l[G], acc[G][VE];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    m[j] = -INFINITY;
+    l[j] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VE; ++e) acc[j][e] = 0.f;
+  }
+
+  // The trip count is uniform across the CTA (every lane takes part in the
+  // shuffles below); rows past the chunk are masked instead.
+  for (int base = 0; base < nrows; base += NG * U) {
+    int4 kr[U], vr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int row = base + u * NG + grp;
+      if (row < nrows) {
+        int slot = slot0 + row;
+        if (slot >= C) slot -= C;
+        kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
+        vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
+      } else {
+        kr[u] = make_int4(0, 0, 0, 0);
+        vr[u] = make_int4(0, 0, 0, 0);
+      }
+    }
+    float sv[G][U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float kf[VE];
+      Vec16<T>::cvt(kr[u], kf);
+      const int row = base + u * NG + grp;
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) dot = fmaf(qf[j][e], kf[e], dot);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        sv[j][u] = (row < nrows && w0 + row >= e0[j]) ? dot : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      float bmax = m[j];
+#pragma unroll
+      for (int u = 0; u < U; ++u) bmax = fmaxf(bmax, sv[j][u]);
+      if (bmax > m[j]) {                               // uniform across the group's lanes
+        const float corr = exp2f(m[j] - bmax);         // 0 when m = -inf
+        l[j] *= corr;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) acc[j][e] *= corr;
+        m[j] = bmax;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float vf[VE];
+      Vec16<T>::cvt(vr[u], vf);
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        // a head that has seen no row yet keeps m = -inf: p = 0, not NaN
+        const float pu = exp2f(sv[j][u] - (m[j] == -INFINITY ? 0.f : m[j]));
+        l[j] += pu;
+#pragma unroll
+        for (int e = 0; e < VE; ++e) acc[j][e] = fmaf(pu, vf[e], acc[j][e]);
+      }
+    }
+  }
+
+  // per head: merge the row groups (log-sum-exp) and write the split's partial
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+#pragma unroll
+    for (int e = 0; e < VE; ++e) g_acc[grp][li * VE + e] = acc[j][e];
+    if (li == 0) {
+      g_m[grp] = m[j];
+      g_l[grp] = l[j];
+    }
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) M = fmaxf(M, g_m[k]);
+    float L = 0.f, od = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        const float w = exp2f(g_m[k] - M);
+        L = fmaf(w, g_l[k], L);
+        if (tid < D) od = fmaf(w, g_acc[k][tid], od);
+      }
+    }
+    const int h = g * G + j;
+    if (nsplit == 1) {
+      if (tid < D)
+        Vec16<T>::store(reinterpret_cast<T*>(p.o) + ((size_t)b * p.Hq + h) * D + tid, L > 0.f ? od / L : 0.f);
+    } else {
+      const size_t idx = (size_t)b * p.hslot_pre[p.Hq] + p.hslot_pre[h] + s;
+      if (tid < D) p.part_o[idx * D + tid] = od;
+      if (tid == 0) {
+        p.part_ml[2 * idx] = M;
+        p.part_ml[2 * idx + 1] = L;
+      }
+    }
+    __syncthreads();                                   // g_acc is reused by the next head
+  }
+  if (nsplit == 1) {
+    if (tid == 0 && W == 0) atomicOr(p.err, kErrEmpty);
+    return;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(&p.ctr[(size_t)b * p.Hq + g], 1u);
+    last_flag = (prev == (unsigned)(nsplit - 1));
+  }
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+#pragma unroll 1
+  for (int j = 0; j < G; ++j) {
+    const int h = g * G + j;
+    const size_t first = (size_t)b * p.hslot_pre[p.Hq] + p.hslot_pre[h];
+    float MM = -INFINITY;
+    for (int ss = 0; ss < nsplit; ++ss) MM = fmaxf(MM, __ldcg(&p.part_ml[2 * (first + ss)]));
+    float LL = 0.f, A = 0.f;
+    if (MM != -INFINITY) {
+      for (int ss = 0; ss < nsplit; ++ss) {
+        const float ms = __ldcg(&p.part_ml[2 * (first + ss)]);
+        const float w = exp2f(ms - MM);              // 0 for splits outside this head's window
+        LL = fmaf(w, __ldcg(&p.part_ml[2 * (first + ss) + 1]), LL);
+        if (tid < D) A = fmaf(w, __ldcg(&p.part_o[(first + ss) * D + tid]), A);
+      }
+    }
+    if (tid < D) Vec16<T>::store(reinterpret_cast<T*>(p.o) + ((size_t)b * p.Hq + h) * D + tid, LL > 0.f ? A / LL : 0.f);
+  }
+  if (tid == 0) {
+    p.ctr[(size_t)b * p.Hq + g] = 0u;
+    if (W == 0) atomicOr(p.err, kErrEmpty);
+  }
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_group(const DecodeParams& p, unsigned grid, cudaStream_t s) {
+  decode_group_kernel<T, D, G><<<grid, kDecThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_group_g(const DecodeParams& p, int G, unsigned grid, cudaStream_t s) {
+  return G == 4 ? launch_group<T, D, 4>(p, grid, s) : launch_group<T, D, 8>(p, grid, s);
+}
+
 template <typename T, int D>
 cudaError_t launch_one(const DecodeParams& p, unsigned grid, cudaStream_t s) {
   decode_kernel<T, D><<<grid, kDecThreads, 0, s>>>(p);
@@ -248,16 +472,24 @@ struct DecodeLayout {
   size_t ctr_off, ml_off, o_off, total;
 };
 
+// Partial slots per sequence: the per-head kernel uses sum_h ceil(S_h / chunk),
+// the group kernel sum_h ceil(C_g(h) / chunk); both are at most
+// Hq * ceil(max_h S_h / chunk), which sizes the workspace without knowing the
+// number of KV heads.
 DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* spans) {
   DecodeLayout L;
-  int items = 0;
-  for (int h = 0; h < Hq; ++h) items += (spans[h] + kChunk - 1) / kChunk;
+  int items = 0, max_s = 0;
+  for (int h = 0; h < Hq; ++h) {
+    items += (spans[h] + kChunk - 1) / kChunk;
+    max_s = max_s > spans[h] ? max_s : spans[h];
+  }
   L.items_per_b = items;
+  const size_t slots = (size_t)Hq * ((max_s + kChunk - 1) / kChunk);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   L.ctr_off = 256;
   L.ml_off = L.ctr_off + up((size_t)B * Hq * 4);
-  L.o_off = L.ml_off + up((size_t)B * items * 2 * 4);
-  L.total = L.o_off + up((size_t)B * items * d * 4);
+  L.o_off = L.ml_off + up((size_t)B * slots * 2 * 4);
+  L.total = L.o_off + up((size_t)B * slots * d * 4);
   return L;
 }
 
@@ -294,6 +526,39 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
     p.goff[g] = c->goff[g];
+  }
+  // The group kernel reads each cached row once for all G heads but does G
+  // dot products and softmax updates per row; the per-head kernel reads
+  // overlapping windows once per head and L2 serves most of the repeats.  On
+  // a Llama3-8B-shaped layer (B=32, 32 query / 8 KV heads, context 8192) the
+  // group kernel was 5 % faster when the heads' windows summed to 2.24x the
+  // group windows and 8 % slower at 2.0x, so it is taken above 2.2x.
+  const int G = Hq / c->Hkv;
+  int64_t head_rows = 0, group_rows = 0;
+  for (int h = 0; h < Hq; ++h) head_rows += spans[h];
+  for (int g = 0; g < c->Hkv; ++g) group_rows += c->cap[g];
+  if ((G == 4 || G == 8) && head_rows * 10 > group_rows * 22) {
+    // group kernel: splits per KV group over its capacity, G partial slots each
+    int items = 0;
+    p.split_pre[0] = 0;
+    p.hslot_pre[0] = 0;
+    for (int g = 0; g < c->Hkv; ++g) {
+      const int ns = (c->cap[g] + kChunk - 1) / kChunk;
+      p.split_pre[g + 1] = p.split_pre[g] + ns;
+      for (int j = 0; j < G; ++j) p.hslot_pre[g * G + j + 1] = p.hslot_pre[g * G + j] + ns;
+      items += ns;
+    }
+    p.items_per_b = items;
+    const long long grid = (long long)c->B * items;
+    if (grid > 0x7fffffffLL) return MOA_ERR_UNSUPPORTED;
+    cudaError_t e;
+    if (c->dtype == MOA_BF16)
+      e = c->d == 128 ? launch_group_g<__nv_bfloat16, 128>(p, G, (unsigned)grid, s)
+                      : launch_group_g<__nv_bfloat16, 64>(p, G, (unsigned)grid, s);
+    else
+      e = c->d == 128 ? launch_group_g<float, 128>(p, G, (unsigned)grid, s)
+                      : launch_group_g<float, 64>(p, G, (unsigned)grid, s);
+    return e == cudaSuccess ? MOA_OK : cuda_fail(e, "decode launch");
   }
   const long long grid = (long long)c->B * L.items_per_b;
   if (grid > 0x7fffffffLL) return MOA_ERR_UNSUPPORTED;

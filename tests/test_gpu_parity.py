@@ -210,6 +210,11 @@ DECODE_CASES = [
     (2, 4, 4, 900, [1, 256, 257, 900], 3),         # multi-split heads, single-split heads
     (3, 8, 2, 50, [40, 7, 64, 64, 300, 1, 299, 17], 4),  # prefix shorter than spans, GQA
     (1, 4, 1, 2000, [1000, 513, 2000, 1], 2),       # window smaller than ring: wraps
+    (2, 8, 4, 700, [700, 1, 300, 513, 64, 65, 2, 699], 3),     # 2 query heads per KV head
+    # windows of a group overlapping enough (sum > 2.2x the group window) for the group-shared kernel
+    (3, 8, 2, 50, [40, 38, 64, 64, 300, 299, 299, 280], 3),
+    (1, 16, 2, 1500, [1500, 3, 700, 701, 64, 1, 1499, 900,     # 8 query heads per KV head
+                      2, 1000, 1024, 513, 257, 5, 1200, 40], 2),
 ]
 
 
@@ -279,13 +284,55 @@ def test_bf16_decode_vicuna7b_layer_full_size_sampled():
         assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
 
 
-def test_decode_empty_sequence_sets_error_bit():
-    B, H, d = 2, 2, 128
-    cache = moa.KVCache(B, H, d, "bf16", [8, 8])
-    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, [8, 8])
+def test_bf16_decode_llama3_gqa_layer_full_size_sampled():
+    """A Llama3-8B-shaped GQA decode layer: B=4, 32 query heads on 8 KV heads, context 8192,
+    per-head spans at 50% density (heterogeneous within each group), one appended token."""
+    B, Hq, Hkv, d, N = 4, 32, 8, 128, 8192
+    a, b = inputs.tables_7b(1001, Hq, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    caps = okv.group_capacities(spans, Hkv)
+    G = Hq // Hkv
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    data = cache.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(15, (data.numel(),)))
+    cache.set_positions([N] * B)
+    rng = np.random.default_rng(4)
+    picks = [(int(rng.integers(B)), int(rng.integers(Hq))) for _ in range(24)] + [(0, 0), (B - 1, Hq - 1)]
+    host = cache.data_bytes().cpu().numpy().tobytes()
+    blocks = {}
+    for bb, hh in picks:
+        if (bb, hh // G) not in blocks:
+            blocks[(bb, hh // G)] = okv.block_from_image(host, bb, hh // G, B, Hkv, d, caps, "bf16")
+    scale = 1.0 / math.sqrt(d)
+    qt = inputs.randn_cuda(16, (B, Hq, d))
+    kt = inputs.randn_cuda(17, (B, Hkv, 1, d))
+    vt = inputs.randn_cuda(18, (B, Hkv, 1, d))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    cache.append(kt, vt)
+    ot = _nan_like((B, Hq, d), torch.bfloat16)
+    moa.moa_decode(cache.handle, qt, ot, Hq, spans, scale, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    assert cache.positions() == [N + 1] * B
+    kt64, vt64, qt64, ot64 = (inputs.as_f64(x) for x in (kt, vt, qt, ot))
+    for bb, hh in picks:
+        g = hh // G
+        K, V = (x.copy() for x in blocks[(bb, g)])
+        C = caps[g]
+        K[N % C] = kt64[bb, g, 0]           # the appended token's slot
+        V[N % C] = vt64[bb, g, 0]
+        ref = okv.decode_row_from_ring(K, V, N + 1, spans[hh], qt64[bb, hh], scale)
+        assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
+
+
+@pytest.mark.parametrize("H,Hkv", [(2, 2), (4, 1)], ids=["mha", "gqa"])
+def test_decode_empty_sequence_sets_error_bit(H, Hkv):
+    B, d = 2, 128
+    spans = [8] * H
+    cache = moa.KVCache(B, Hkv, d, "bf16", [8] * Hkv)
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, spans)
     q = inputs.randn_cuda(1, (B, H, d))
     o = _nan_like((B, H, d), torch.bfloat16)
-    moa.moa_decode(cache.handle, q, o, H, [8, 8], 0.1, ws.ptr, ws.nbytes)
+    moa.moa_decode(cache.handle, q, o, H, spans, 0.1, ws.ptr, ws.nbytes)
     with pytest.raises(moa.MoaError) as e:
         cache.positions()
     assert e.value.status == moa.MOA_ERR_INVALID_ARG
