@@ -56,7 +56,8 @@ def _peaks():
 
 def _workload_desc():
     return ("vicuna7b-shaped: prefill B=%d H=%d d=%d N=%d density %.2f + decode %dL x %dH B=%d d=%d ctx %d "
-            "density %.2f" % (P_B, P_H, P_D, P_N, P_DENSITY, D_L, D_H, D_B, D_D, D_N, D_DENSITY))
+            "density %.2f (append and attend fused per layer)"
+            % (P_B, P_H, P_D, P_N, P_DENSITY, D_L, D_H, D_B, D_D, D_N, D_DENSITY))
 
 
 def _config():
@@ -247,9 +248,11 @@ def run_ours(args):
         d_o.append(torch.empty((D_B, D_H, D_D), dtype=torch.bfloat16, device=dev))
     torch.cuda.synchronize()
     d_scale = 1.0 / math.sqrt(D_D)
-    kv_bytes_layer = [D_B * sum(2 * S * D_D * 2 for S in sp) + 2 * D_B * D_H * D_D * 2 for sp in d_spans]
+    # K/V windows read, q read and o written, and the new token's k, v read and written to the cache
+    kv_bytes_layer = [D_B * sum(2 * S * D_D * 2 for S in sp) + 2 * D_B * D_H * D_D * 2 + 4 * D_B * D_H * D_D * 2
+                      for sp in d_spans]
     kv_bytes_step = sum(kv_bytes_layer)
-    launches_per_step = 2 + 2 * D_L
+    launches_per_step = 2 + D_L
 
     def step(ev):
         # rule evaluation for the prompt (host), prefill, cache fill, decode step
@@ -261,10 +264,9 @@ def run_ours(args):
         moa.moa_kv_append(p_cache.handle, k, v, P_N, stream)
         ev["d0"].record(stream)
         for layer in range(D_L):
-            moa.moa_kv_append(caches[layer].handle, d_k[layer], d_v[layer], 1, stream)
             ev["k0"][layer].record(stream)
-            moa.moa_decode(caches[layer].handle, d_q[layer], d_o[layer], D_H, d_spans[layer], d_scale,
-                           d_ws[layer].ptr, d_ws[layer].nbytes, stream)
+            moa.moa_decode_append(caches[layer].handle, d_q[layer], d_k[layer], d_v[layer], d_o[layer], D_H,
+                                  d_spans[layer], d_scale, d_ws[layer].ptr, d_ws[layer].nbytes, stream)
             ev["k1"][layer].record(stream)
         ev["d1"].record(stream)
 
@@ -332,9 +334,8 @@ def run_ours(args):
             e_q[layer].copy_(h_q[layer], non_blocking=True)
             e_k[layer].copy_(h_k[layer], non_blocking=True)
             e_v[layer].copy_(h_v[layer], non_blocking=True)
-            moa.moa_kv_append(caches[layer].handle, e_k[layer], e_v[layer], 1, stream)
-            moa.moa_decode(caches[layer].handle, e_q[layer], d_o[layer], D_H, d_spans[layer], d_scale,
-                           d_ws[layer].ptr, d_ws[layer].nbytes, stream)
+            moa.moa_decode_append(caches[layer].handle, e_q[layer], e_k[layer], e_v[layer], d_o[layer], D_H,
+                                  d_spans[layer], d_scale, d_ws[layer].ptr, d_ws[layer].nbytes, stream)
             h_o[layer].copy_(d_o[layer], non_blocking=True)
 
     for _ in range(2):
@@ -370,7 +371,8 @@ def run_ours(args):
             "config": _config(),
             "kv_gbs": round(kv_gbs, 2),
             "decode_ms_per_step": round(decode_ms, 4),
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel<bf16,128> (moa_decode, one layer)",
+            "roofline": {"bound": "hbm",
+                         "kernel": "decode_kernel<bf16,128> (moa_decode_append: one layer, append + attend)",
                          "achieved": round(dec_achieved, 2), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(dec_achieved / hbm_peak, 4), "peak_kind": peak_kind + " copy (hbm_gbs)",
                          "frac_of_nominal": round(dec_achieved / NOMINAL_HBM_GBS, 4),
@@ -528,8 +530,7 @@ def run_profile_case(case, launches=3):
         v = inputs.randn_cuda(400, (D_B, D_H, 1, D_D))
         o = torch.empty_like(q)
         for _ in range(launches):
-            moa.moa_kv_append(c.handle, k, v, 1)
-            moa.moa_decode(c.handle, q, o, D_H, sp, 1.0 / math.sqrt(D_D), ws.ptr, ws.nbytes)
+            moa.moa_decode_append(c.handle, q, k, v, o, D_H, sp, 1.0 / math.sqrt(D_D), ws.ptr, ws.nbytes)
         c.positions()
     torch.cuda.synchronize()
     print("profile case %s done" % case)

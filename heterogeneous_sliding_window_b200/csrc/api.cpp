@@ -222,6 +222,23 @@ extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, v
   return launch_append(fill, k, v, (int32_t)N, s);
 }
 
+extern "C" moa_status moa_decode_append(moa_kv_cache* c, const void* q, const void* k, const void* v,
+                                        void* o, int32_t Hq, const int32_t* spans, float scale, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  if (!c || !q || !k || !v || !o || !spans) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if (Hq < 1 || Hq > MOA_MAX_HEADS || Hq % c->Hkv != 0) return MOA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
+  const int32_t G = Hq / c->Hkv;
+  for (int32_t h = 0; h < Hq; ++h) {
+    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+    if (spans[h] > c->cap[h / G]) return MOA_ERR_CAPACITY;
+  }
+  if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
+  if (ws_bytes < decode_workspace_bytes(c->B, Hq, c->d, spans)) return MOA_ERR_WORKSPACE;
+  return launch_decode(c, q, o, Hq, spans, scale, ws, ws_bytes, (cudaStream_t)stream, k, v);
+}
+
 extern "C" moa_status moa_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                                  const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                  void* stream) {

@@ -31,8 +31,11 @@ constexpr int kChunk = 512;          // window entries per split
 constexpr int kUnroll = 8;           // rows per batch: 2*kUnroll 16-byte loads in flight
 
 struct DecodeParams {
-  const char* data;                  // cache data region
-  const int64_t* t;                  // cache header: tokens per sequence
+  char* data;                        // cache data region
+  int64_t* t;                        // cache header: tokens per sequence
+  const void* k_new;                 // fused append: the step's k, v [B, Hkv, 1, D]; null otherwise
+  const void* v_new;
+  uint32_t* bctr;                    // fused append: CTAs of sequence b that have read t[b]
   uint32_t* err;                     // cache header: error word
   const void* q;
   void* o;
@@ -71,6 +74,22 @@ template <> struct Vec16<__nv_bfloat16> {
   __device__ static void store(__nv_bfloat16* dst, float x) { *dst = __float2bfloat16_rn(x); }
 };
 
+// Fused append: every CTA of sequence b counts itself once all its threads
+// have read t[b]; the last of the items_per_b CTAs sets t[b] to t0 + 1 (no
+// CTA of this launch reads t[b] after that) and rearms the counter.
+__device__ __forceinline__ void step_counted(const DecodeParams& p, int b, int64_t t0) {
+  (void)t0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(&p.bctr[b], 1u);
+    if (prev == (unsigned)(p.items_per_b - 1)) {
+      p.bctr[b] = 0u;
+      p.t[b] = t0 + 1;
+    }
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int VE = Vec16<T>::N;     // elements per 16-byte vector
@@ -101,15 +120,24 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   const int nsplit = p.split_pre[h + 1] - p.split_pre[h];
   const int g = h / p.G;
   const int C = p.cap[g];
-  const int64_t tb = p.t[b];
+  const bool fused = p.k_new != nullptr;
+  const int64_t t0 = p.t[b];
+  if (fused) step_counted(p, b, t0);
+  const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int Seff = (int)(tb < (int64_t)p.span[h] ? tb : (int64_t)p.span[h]);
   const int w0 = s * kChunk;
   const int nrows = max(0, min(kChunk, Seff - w0));
   const int64_t pos0 = tb - Seff + w0;                 // first window position of this split
   const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
 
-  const T* Kb = reinterpret_cast<const T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
-  const T* Vb = Kb + (size_t)C * D;
+  T* Kb = reinterpret_cast<T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
+  T* Vb = Kb + (size_t)C * D;
+  // fused append: the newest window entry comes from the step's k, v, and the
+  // group's first head writes it to its slot
+  const int e_new = fused ? Seff - 1 : -1;
+  const bool writer = fused && h == g * p.G;
+  const T* kn = fused ? reinterpret_cast<const T*>(p.k_new) + ((size_t)b * (p.Hq / p.G) + g) * D : nullptr;
+  const T* vn = fused ? reinterpret_cast<const T*>(p.v_new) + ((size_t)b * (p.Hq / p.G) + g) * D : nullptr;
 
   float qf[VE];
   {
@@ -135,8 +163,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       if (row < nrows) {
         int slot = slot0 + row;
         if (slot >= C) slot -= C;
-        kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
-        vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
+        if (w0 + row == e_new) {
+          kr[u] = __ldg(reinterpret_cast<const int4*>(kn + li * VE));
+          vr[u] = __ldg(reinterpret_cast<const int4*>(vn + li * VE));
+          if (writer) {
+            *reinterpret_cast<int4*>(Kb + (size_t)slot * D + li * VE) = kr[u];
+            *reinterpret_cast<int4*>(Vb + (size_t)slot * D + li * VE) = vr[u];
+          }
+        } else {
+          kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
+          vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
+        }
       } else {
         kr[u] = make_int4(0, 0, 0, 0);
         vr[u] = make_int4(0, 0, 0, 0);
@@ -282,15 +319,23 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
   const int s = r - p.split_pre[g];
   const int nsplit = p.split_pre[g + 1] - p.split_pre[g];
   const int C = p.cap[g];
-  const int64_t tb = p.t[b];
+  const bool fused = p.k_new != nullptr;
+  const int64_t t0 = p.t[b];
+  if (fused) step_counted(p, b, t0);
+  const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);   // the group's longest window
   const int w0 = s * kChunk;
   const int nrows = max(0, min(kChunk, W - w0));
   const int64_t pos0 = tb - W + w0;
   const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
 
-  const T* Kb = reinterpret_cast<const T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
-  const T* Vb = Kb + (size_t)C * D;
+  T* Kb = reinterpret_cast<T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
+  T* Vb = Kb + (size_t)C * D;
+  // fused append: the newest window entry comes from the step's k, v, which
+  // this CTA (the group's only reader of that entry) writes to its slot
+  const int e_new = fused ? W - 1 : -1;
+  const T* kn = fused ? reinterpret_cast<const T*>(p.k_new) + ((size_t)b * Hkv + g) * D : nullptr;
+  const T* vn = fused ? reinterpret_cast<const T*>(p.v_new) + ((size_t)b * Hkv + g) * D : nullptr;
 
   // head j of the group sees window entries e >= e0[j] (e counts from the
   // oldest entry of the group's window)
@@ -327,8 +372,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
       if (row < nrows) {
         int slot = slot0 + row;
         if (slot >= C) slot -= C;
-        kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
-        vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
+        if (w0 + row == e_new) {
+          kr[u] = __ldg(reinterpret_cast<const int4*>(kn + li * VE));
+          vr[u] = __ldg(reinterpret_cast<const int4*>(vn + li * VE));
+          *reinterpret_cast<int4*>(Kb + (size_t)slot * D + li * VE) = kr[u];
+          *reinterpret_cast<int4*>(Vb + (size_t)slot * D + li * VE) = vr[u];
+        } else {
+          kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
+          vr[u] = __ldcs(reinterpret_cast<const int4*>(Vb + (size_t)slot * D + li * VE));
+        }
       } else {
         kr[u] = make_int4(0, 0, 0, 0);
         vr[u] = make_int4(0, 0, 0, 0);
@@ -469,7 +521,7 @@ cudaError_t launch_one(const DecodeParams& p, unsigned grid, cudaStream_t s) {
 
 struct DecodeLayout {
   int items_per_b;
-  size_t ctr_off, ml_off, o_off, total;
+  size_t ctr_off, bctr_off, ml_off, o_off, total;
 };
 
 // Partial slots per sequence: the per-head kernel uses sum_h ceil(S_h / chunk),
@@ -487,7 +539,8 @@ DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* span
   const size_t slots = (size_t)Hq * ((max_s + kChunk - 1) / kChunk);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   L.ctr_off = 256;
-  L.ml_off = L.ctr_off + up((size_t)B * Hq * 4);
+  L.bctr_off = L.ctr_off + up((size_t)B * Hq * 4);
+  L.ml_off = L.bctr_off + up((size_t)B * 4);
   L.o_off = L.ml_off + up((size_t)B * slots * 2 * 4);
   L.total = L.o_off + up((size_t)B * slots * d * 4);
   return L;
@@ -500,17 +553,21 @@ size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* s
 }
 
 moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, const int32_t* spans,
-                         float scale, void* ws, size_t ws_bytes, cudaStream_t s) {
+                         float scale, void* ws, size_t ws_bytes, cudaStream_t s, const void* k_new,
+                         const void* v_new) {
   const DecodeLayout L = decode_layout(c->B, Hq, c->d, spans);
   if (ws_bytes < L.total) return MOA_ERR_WORKSPACE;
   DecodeParams p;
   p.data = c->buf + c->header;
-  p.t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
+  p.t = reinterpret_cast<int64_t*>(c->buf + kHdrT);
+  p.k_new = k_new;
+  p.v_new = v_new;
   p.err = reinterpret_cast<uint32_t*>(c->buf + kHdrErr);
   p.q = q;
   p.o = o;
   char* w = (char*)ws;
   p.ctr = reinterpret_cast<uint32_t*>(w + L.ctr_off);
+  p.bctr = reinterpret_cast<uint32_t*>(w + L.bctr_off);
   p.part_ml = reinterpret_cast<float*>(w + L.ml_off);
   p.part_o = reinterpret_cast<float*>(w + L.o_off);
   p.Hq = Hq;

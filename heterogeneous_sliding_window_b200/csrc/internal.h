@@ -54,7 +54,7 @@ moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t 
 size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans);
 moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                          const int32_t* spans, float scale, void* ws, size_t ws_bytes,
-                         cudaStream_t s);
+                         cudaStream_t s, const void* k_new = nullptr, const void* v_new = nullptr);
 
 // prefill_simt.cu (fp32)
 moa_status launch_prefill_f32(const float* q, const float* k, const float* v, float* o,

@@ -24,7 +24,7 @@ EXPORTS = (
     "moa_status_string", "moa_rules_eval", "moa_kv_bytes", "moa_kv_header_bytes", "moa_kv_alloc",
     "moa_kv_free", "moa_kv_append", "moa_kv_positions", "moa_kv_set_positions", "moa_kv_layout",
     "moa_workspace_bytes", "moa_workspace_init", "moa_workspace_check", "moa_prefill",
-    "moa_prefill_schedule", "moa_decode", "moa_decode_static_ws",
+    "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws",
 )
 
 
@@ -65,6 +65,7 @@ def load():
                                        vp, sz, vp, vp]),
         "moa_prefill_schedule": (ctypes.c_int, [i32, i32, i64, P(i32), i32, P(i32), i64, P(i64)]),
         "moa_decode": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
+        "moa_decode_append": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_static_ws": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp]),
     }
     for name, (res, args) in sig.items():
@@ -220,6 +221,12 @@ def moa_decode(handle, q, o, Hq, spans, scale, ws, ws_bytes, stream=None):
     sp, spp = _i32(spans)
     _check(load().moa_decode(handle, _ptr(q), _ptr(o), Hq, spp, float(scale), _ptr(ws), ws_bytes,
                              _stream(stream)), "moa_decode")
+
+
+def moa_decode_append(handle, q, k, v, o, Hq, spans, scale, ws, ws_bytes, stream=None):
+    sp, spp = _i32(spans)
+    _check(load().moa_decode_append(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), Hq, spp, float(scale), _ptr(ws),
+                                    ws_bytes, _stream(stream)), "moa_decode_append")
 
 
 def moa_decode_static_ws(handle, q, o, Hq, spans, scale, stream=None):

@@ -197,6 +197,18 @@ moa_status moa_decode(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
                       const int32_t* spans, float scale, void* workspace, size_t ws_bytes,
                       void* stream);
 
+/* One decode step in one launch: the same result, cache bytes and positions as
+ * moa_kv_append(cache, k, v, 1) followed by moa_decode(cache, q, o, ...)
+ * ("Mixture of Attention" project page, "Demo" step 03: the fixed-size
+ * per-head cache is written at slot t mod C_g and each head attends to its
+ * last S_h positions).  k, v: [B, Hkv, 1, d] device, 16-byte aligned.  The
+ * window entry of the new token is taken from k, v directly; one CTA per
+ * (sequence, kv head) writes it to its slot, and the last CTA of each
+ * sequence to have read t_b advances it.  Workspace and errors as moa_decode. */
+moa_status moa_decode_append(moa_kv_cache* cache, const void* q, const void* k, const void* v,
+                             void* o, int32_t Hq, const int32_t* spans, float scale,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Decode without a caller workspace.  The paper has no counterpart: this is
  * a deployment convenience of this library.

@@ -246,6 +246,58 @@ def test_bf16_decode_matches_oracle(case):
     assert cache.positions() == ring.t
 
 
+FUSED_CASES = [
+    # (B, Hq, Hkv, dtype, d, prefix, spans, steps)
+    (2, 4, 4, "bf16", 128, 900, [1, 256, 257, 900], 3),                    # per-head kernel
+    (3, 8, 2, "bf16", 128, 50, [40, 7, 64, 64, 300, 1, 299, 17], 4),       # GQA, per-head kernel
+    (3, 8, 2, "bf16", 128, 50, [40, 38, 64, 64, 300, 299, 299, 280], 3),   # GQA, group kernel
+    (1, 16, 2, "bf16", 128, 1500, [1500, 3, 700, 701, 64, 1, 1499, 900,
+                                   2, 1000, 1024, 513, 257, 5, 1200, 40], 2),  # 8 heads per group
+    (1, 4, 1, "bf16", 128, 2000, [1000, 513, 2000, 1], 2),                 # ring wraps
+    (2, 4, 2, "f32", 64, 0, [1, 5, 32, 17], 40),                           # from an empty cache
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "B%d_H%d_%d_%s_T%d" % (c[0], c[1], c[2], c[3], c[5]))
+def test_decode_append_equals_append_then_decode(case):
+    """moa_decode_append gives, bit for bit, the outputs, cache bytes and positions of
+    moa_kv_append followed by moa_decode, and matches the oracle."""
+    B, Hq, Hkv, dt, d, prefix, spans, steps = case
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    tol = BF16_TOL if dt == "bf16" else F32_TOL
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    two = moa.KVCache(B, Hkv, d, dt, caps)
+    one = moa.KVCache(B, Hkv, d, dt, caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    if prefix:
+        k0 = inputs.randn(72, (B, Hkv, prefix, d), dt)
+        v0 = inputs.randn(73, (B, Hkv, prefix, d), dt)
+        for c in (two, one):
+            c.append(k0.to(DEV), v0.to(DEV))
+        ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+    ws2 = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    ws1 = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    for step in range(steps):
+        qt = inputs.randn(82 + step, (B, Hq, d), dt)
+        kt = inputs.randn(92 + step, (B, Hkv, 1, d), dt)
+        vt = inputs.randn(97 + step, (B, Hkv, 1, d), dt)
+        ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+        o2 = _nan_like((B, Hq, d), tdt)
+        o1 = _nan_like((B, Hq, d), tdt)
+        two.append(kt.to(DEV), vt.to(DEV))
+        moa.moa_decode(two.handle, qt.to(DEV), o2, Hq, spans, scale, ws2.ptr, ws2.nbytes)
+        moa.moa_decode_append(one.handle, qt.to(DEV), kt.to(DEV), vt.to(DEV), o1, Hq, spans, scale,
+                              ws1.ptr, ws1.nbytes)
+        torch.cuda.synchronize()
+        assert torch.equal(o1.view(torch.int16 if dt == "bf16" else torch.int32),
+                           o2.view(torch.int16 if dt == "bf16" else torch.int32)), step
+        assert torch.equal(one.data_bytes(), two.data_bytes()), step
+        ref = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+        assert np.max(np.abs(inputs.as_f64(o1) - ref)) <= tol, step
+    assert one.positions() == two.positions() == ring.t
+
+
 def test_bf16_decode_vicuna7b_layer_full_size_sampled():
     """One layer of the decode workload: B=32, 32 heads, context 4096, 50% density."""
     B, H, d, N = 32, 32, 128, 4096
