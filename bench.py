@@ -127,6 +127,24 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of per-rank timings (ms) over all ranks; every rank gets the result.
+
+    With one process (dist None) the values come back unchanged.  The slowest rank's device time
+    is the job's time: throughput is the units all ranks processed divided by it.
+    """
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank, n_ranks, max_ms):
+    """Whole-job units per second: every rank processes units_per_rank in max_ms (the slowest rank)."""
+    return n_ranks * units_per_rank / (max_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reported baseline, never the product path)
 # ---------------------------------------------------------------------------
@@ -307,13 +325,11 @@ def run_ours(args):
     for c in caches:
         c.positions()
 
-    vals = torch.tensor([total_ms, prefill_ms, decode_ms, dec_kernel_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, prefill_ms, decode_ms, dec_kernel_ms = vals.tolist()
+    total_ms, prefill_ms, decode_ms, dec_kernel_ms = max_over_ranks(
+        [total_ms, prefill_ms, decode_ms, dec_kernel_ms], dist, dev)
     ms_per_step = total_ms / args.steps
 
-    tokens_per_s = ws_n * D_B / (decode_ms * 1e-3)
+    tokens_per_s = job_throughput(D_B, ws_n, decode_ms)
     kv_gbs = ws_n * kv_bytes_step / (decode_ms * 1e-3) / 1e9
     prefill_tflops = ws_n * p_flops / (prefill_ms * 1e-3) / 1e12
     dec_bytes_launch = sum(kv_bytes_layer) / D_L
@@ -350,10 +366,7 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = e2e_ms.item()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dist, dev)[0]
     h2d = sum(x.numel() * x.element_size() for x in h_q + h_k + h_v)
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
@@ -387,7 +400,7 @@ def run_ours(args):
                                      "frac_of_sustained": round(p_achieved / tf_sustained, 4),
                                      "frac_of_nominal": round(p_achieved / NOMINAL_BF16_TFLOPS, 4),
                                      "traffic": traffic.get("prefill")}},
-            "e2e": {"value": round(ws_n * D_B / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+            "e2e": {"value": round(job_throughput(D_B, ws_n, e2e_ms), 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "note": "decode step through the C ABI from pinned host q/k/v to host o"},
             "gqa_decode": gqa,

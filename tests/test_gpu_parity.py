@@ -172,6 +172,73 @@ def test_bf16_prefill_vicuna7b_full_size_sampled():
     assert np.max(np.abs(got - ref)) <= BF16_TOL
 
 
+def test_bf16_prefill_vicuna13b_mixed_spans_sampled():
+    """A Vicuna-13B-shaped layer: B=1, 40 heads, d=128, N=16384, fixed-local heads mixed with
+    elastic heads at 50% density (config 4), sampled rows."""
+    B, H, N, d = 1, 40, 16384, 128
+    a, b = inputs.tables_13b_mix(5, H, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    assert spans == orules.eval_spans(a, b, N, 64)
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(21, (B, H, N, d))
+    k = inputs.randn_cuda(22, (B, H, N, d))
+    v = inputs.randn_cuda(23, (B, H, N, d))
+    o = _bf16_prefill(q, k, v, spans, scale)
+    assert not torch.isnan(o).any()
+    rows = _sample_rows(B, H, N, np.random.default_rng(1), n=64)
+    rows = [r for r in rows if r[1] % 5 == 0 or r[2] in (N - 1,)][:120]
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale, rows=rows)
+    got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
+    assert np.max(np.abs(got - ref)) <= BF16_TOL
+
+
+def test_decode_append_replayed_from_cuda_graph():
+    """Two layers of moa_decode_append captured once in a CUDA graph and replayed for four
+    steps (new q, k, v copied into the captured buffers each time) match the oracle."""
+    B, Hq, Hkv, d, prefix = 2, 8, 2, 128, 300
+    layers = [[300, 7, 64, 64, 250, 1, 299, 17], [40, 38, 64, 64, 300, 299, 299, 280]]
+    scale = 1.0 / math.sqrt(d)
+    state = []
+    for li, spans in enumerate(layers):
+        caps = okv.group_capacities(spans, Hkv)
+        cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+        ring = okv.RingCache(B, Hkv, d, caps)
+        k0 = inputs.randn(110 + li, (B, Hkv, prefix, d))
+        v0 = inputs.randn(120 + li, (B, Hkv, prefix, d))
+        cache.append(k0.to(DEV), v0.to(DEV))
+        ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+        ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+        bufs = [torch.zeros((B, Hq, d), dtype=torch.bfloat16, device=DEV),
+                torch.zeros((B, Hkv, 1, d), dtype=torch.bfloat16, device=DEV),
+                torch.zeros((B, Hkv, 1, d), dtype=torch.bfloat16, device=DEV),
+                torch.zeros((B, Hq, d), dtype=torch.bfloat16, device=DEV)]
+        state.append((spans, cache, ring, ws, bufs))
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for spans, cache, ring, ws, (q, k, v, o) in state:
+            moa.moa_decode_append(cache.handle, q, k, v, o, Hq, spans, scale, ws.ptr, ws.nbytes, stream)
+    torch.cuda.synchronize()
+    for step in range(4):
+        host = []
+        for li, (spans, cache, ring, ws, (q, k, v, o)) in enumerate(state):
+            qt = inputs.randn(130 + 10 * step + li, (B, Hq, d))
+            kt = inputs.randn(170 + 10 * step + li, (B, Hkv, 1, d))
+            vt = inputs.randn(210 + 10 * step + li, (B, Hkv, 1, d))
+            q.copy_(qt)
+            k.copy_(kt)
+            v.copy_(vt)
+            ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+            host.append(qt)
+        graph.replay()
+        torch.cuda.synchronize()
+        for (spans, cache, ring, ws, (q, k, v, o)), qt in zip(state, host):
+            ref = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+            assert np.max(np.abs(inputs.as_f64(o) - ref)) <= BF16_TOL, step
+    for spans, cache, ring, ws, bufs in state:
+        assert cache.positions() == ring.t == [prefix + 4] * B
+
+
 def test_bf16_prefill_llama3_gqa_dense_sampled():
     """Hq=32 / Hkv=8, N=32768, every span = N (the dense causal check), sampled rows."""
     B, Hq, Hkv, N, d = 1, 32, 8, 32768, 128
