@@ -370,6 +370,7 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in h_q + h_k + h_v)
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
+    read_gbs = read_only_gbs([c.data_bytes() for c in caches[:4]], stream)
 
     result = None
     if rank == 0:
@@ -389,6 +390,8 @@ def run_ours(args):
                          "achieved": round(dec_achieved, 2), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(dec_achieved / hbm_peak, 4), "peak_kind": peak_kind + " copy (hbm_gbs)",
                          "frac_of_nominal": round(dec_achieved / NOMINAL_HBM_GBS, 4),
+                         "read_only_gbs": round(read_gbs, 1),
+                         "frac_of_read_only": round(dec_achieved / read_gbs, 4),
                          "traffic": traffic.get("decode"),
                          "algorithmic_bytes_per_launch": int(dec_bytes_launch)},
             "prefill": {"tflops": round(prefill_tflops, 2), "ms": round(prefill_ms, 4),
@@ -414,6 +417,29 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def read_only_gbs(bufs, stream, reps=5):
+    """Read-only HBM roofline measured in this run: libmoa's stream-read probe
+    (16-byte loads on every SM, the decode kernel's access width) over resident
+    decode caches, GB/s of the best of `reps` passes."""
+    import torch
+    from heterogeneous_sliding_window_b200 import moa
+    out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sizes = [b.numel() * b.element_size() // 16 * 16 for b in bufs]
+    for b, n in zip(bufs, sizes):
+        moa.moa_stream_read(b, n, out, stream)
+    best = float("inf")
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for b, n in zip(bufs, sizes):
+            moa.moa_stream_read(b, n, out, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return sum(sizes) / (best * 1e-3) / 1e9
 
 
 def gqa_decode_layer(stream, reps=20):

@@ -173,6 +173,13 @@ extern "C" moa_status moa_workspace_check(const void* ws, void* stream) {
   return err ? MOA_ERR_TIMEOUT : MOA_OK;
 }
 
+extern "C" moa_status moa_stream_read(const void* buf, size_t bytes, void* out, void* stream) {
+  if (!buf || !out || bytes % 16 != 0 || reinterpret_cast<uintptr_t>(buf) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(out) % 8 != 0)
+    return MOA_ERR_INVALID_ARG;
+  return launch_stream_read(buf, bytes, out, (cudaStream_t)stream);
+}
+
 extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
                                            int32_t n_ctas, int32_t* rows_out, int64_t cap,
                                            int64_t* n_rows_out) {

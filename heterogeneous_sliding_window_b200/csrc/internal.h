@@ -47,6 +47,9 @@ inline moa_status check_launch(const char* where) {
 }
 
 // kv.cu
+// Reads `bytes` (a multiple of 16) at 16-byte-aligned `buf` into a checksum
+// at `out` (one uint64 on the device).
+moa_status launch_stream_read(const void* buf, size_t bytes, void* out, cudaStream_t stream);
 moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
                          cudaStream_t s);
 

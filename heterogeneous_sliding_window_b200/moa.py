@@ -24,7 +24,7 @@ EXPORTS = (
     "moa_status_string", "moa_rules_eval", "moa_kv_bytes", "moa_kv_header_bytes", "moa_kv_alloc",
     "moa_kv_free", "moa_kv_append", "moa_kv_positions", "moa_kv_set_positions", "moa_kv_layout",
     "moa_workspace_bytes", "moa_workspace_init", "moa_workspace_check", "moa_prefill",
-    "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws",
+    "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws", "moa_stream_read",
 )
 
 
@@ -67,6 +67,7 @@ def load():
         "moa_decode": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_append": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_static_ws": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp]),
+        "moa_stream_read": (ctypes.c_int, [vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -234,6 +235,11 @@ def moa_decode_static_ws(handle, q, o, Hq, spans, scale, stream=None):
     sp, spp = _i32(spans)
     _check(load().moa_decode_static_ws(handle, _ptr(q), _ptr(o), Hq, spp, float(scale), _stream(stream)),
            "moa_decode_static_ws")
+
+
+def moa_stream_read(buf, nbytes, out, stream=None):
+    """Read-only bandwidth probe: checksum of `nbytes` at `buf` into the device uint64 `out`."""
+    _check(load().moa_stream_read(_ptr(buf), int(nbytes), _ptr(out), _stream(stream)), "moa_stream_read")
 
 
 # ---- conveniences over torch-owned device memory ------------------------------

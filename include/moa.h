@@ -149,6 +149,18 @@ moa_status moa_workspace_init(void* workspace, size_t bytes, void* stream);
  * bounded wait in the last prefill using it gave up, else MOA_OK. */
 moa_status moa_workspace_check(const void* workspace, void* stream);
 
+/* Read-only bandwidth probe for the decode roofline.  Decode attention
+ * reads each head's window of K/V rows once per token and writes almost
+ * nothing, so its bandwidth ceiling is a plain read stream.  Reads `bytes`
+ * of device memory at `buf` once with the decode kernel's access width
+ * (16-byte loads, every SM) and writes their checksum to `out` (device
+ * uint64): with the buffer seen as little-endian uint32 words, the XOR of
+ * the even-indexed words in the high half and of the odd-indexed words in
+ * the low half.  buf must be 16-byte aligned, bytes a multiple of 16, out
+ * 8-byte aligned (else MOA_ERR_INVALID_ARG, nothing launched).  Enqueued on
+ * `stream`; the caller owns both buffers. */
+moa_status moa_stream_read(const void* buf, size_t bytes, void* out, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Prefill: windowed causal attention over a whole prompt ("Finding two" and
  * its N x N causal-band figure; blog section 2.1).  For every (b, h, i):

@@ -183,6 +183,14 @@ def test_prefill_argument_errors_need_no_gpu():
     assert e.value.status == moa.MOA_ERR_UNSUPPORTED
 
 
+def test_stream_read_argument_errors_need_no_gpu():
+    for buf, nbytes, out in [(None, 16, 4096), (4096, 16, None), (4104, 16, 4096), (4096, 24, 4096),
+                             (4096, 16, 4100)]:
+        with pytest.raises(moa.MoaError) as e:
+            moa.moa_stream_read(buf, nbytes, out, 0)
+        assert e.value.status == moa.MOA_ERR_INVALID_ARG, (buf, nbytes, out)
+
+
 def test_workspace_sizes():
     spans = [64, 300, 4096, 1]
     d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)

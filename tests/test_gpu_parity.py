@@ -465,3 +465,21 @@ def test_decode_rejects_span_above_capacity():
     with pytest.raises(moa.MoaError) as e:
         moa.moa_decode(cache.handle, q, q.clone(), 1, [65], 0.1, ws.ptr, ws.nbytes)
     assert e.value.status == moa.MOA_ERR_CAPACITY
+
+
+@pytest.mark.parametrize("nbytes", [0, 16, 48, (64 << 20) + 4096 + 48])
+def test_stream_read_checksum(nbytes):
+    """The read-only bandwidth probe reads every byte once: its checksum is the
+    XOR of the even-indexed 32-bit words (high half) and of the odd-indexed
+    words (low half), recomputed here on the host."""
+    rng = np.random.default_rng(7)
+    host = rng.integers(0, 2 ** 32, size=max(nbytes // 4, 1), dtype=np.uint32)[: nbytes // 4]
+    buf = torch.from_numpy(host.view(np.int32).copy()).to(DEV) if nbytes else torch.empty(4, dtype=torch.int32,
+                                                                                          device=DEV)
+    out = torch.full((1,), -1, dtype=torch.int64, device=DEV)
+    moa.moa_stream_read(buf, nbytes, out)
+    torch.cuda.synchronize()
+    got = int(out.cpu().numpy().view(np.uint64)[0])
+    hi = int(np.bitwise_xor.reduce(host[0::2])) if nbytes else 0
+    lo = int(np.bitwise_xor.reduce(host[1::2])) if nbytes else 0
+    assert got == (hi << 32) | lo
