@@ -89,6 +89,50 @@ def prefill(q, k, v, spans, scale, rows=None):
     return out
 
 
+def chunk(q, k_hist, v_hist, t, spans, scale, rows=None):
+    """Windowed causal attention of a chunk of new tokens that continues each sequence.
+
+    The same definition as ``prefill``, at an offset: query i of sequence b
+    is the token at position P = t[b] + i and attends to window(P, S_h) of
+    that sequence's keys (positions earlier than the chunk included).  This
+    is the prefill of a prompt that arrives in pieces while decoding serves
+    from the fixed-size cache ("Mixture of Attention" project page, "Demo"
+    step 03); with t[b] = 0 it is ``prefill`` of the chunk.
+
+    q: [B, Hq, n, d], queries of positions t[b] .. t[b]+n-1.
+    k_hist, v_hist: per sequence b an array [Hkv, t[b]+n, d] with the keys
+    and values of every position 0 .. t[b]+n-1 (the chunk's own last).
+    t: tokens before the chunk, one per sequence.
+    Returns float64 [B, Hq, n, d], or with ``rows`` ((b, h, i) triples) the
+    float64 [len(rows), d] of those output rows only.
+    """
+    q = np.asarray(q)
+    B, Hq, n, d = q.shape
+    if len(t) != B or len(k_hist) != B or len(v_hist) != B:
+        raise ValueError("one history and one position per sequence")
+    if len(spans) != Hq:
+        raise ValueError("one span per query head")
+    Hkv = np.asarray(k_hist[0]).shape[0]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    for b in range(B):
+        if np.asarray(k_hist[b]).shape[1] != int(t[b]) + n or np.asarray(v_hist[b]).shape != np.asarray(k_hist[b]).shape:
+            raise ValueError("history of sequence %d must hold t[b] + n positions" % b)
+    if rows is None:
+        rows_list = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(n)]
+    else:
+        rows_list = list(rows)
+    out = np.empty((len(rows_list), d), dtype=np.float64)
+    for r, (b, h, i) in enumerate(rows_list):
+        P = int(t[b]) + i
+        lo, hi = window(P, int(spans[h]))
+        out[r] = attend_row(q[b, h, i], k_hist[b][h // G], v_hist[b][h // G], lo, hi, scale)
+    if rows is None:
+        return out.reshape(B, Hq, n, d)
+    return out
+
+
 def in_window_flops(spans, N, d, B=1):
     """Algorithmic FLOPs of prefill counting only in-window work.
 

@@ -159,3 +159,62 @@ def test_in_window_flops_counts_mask_entries():
         for S in spans:
             count += sum(1 for i in range(N) for j in range(N) if j <= i and j > i - S)
         assert attention.in_window_flops(spans, N, d) == 4 * d * count
+
+
+def test_chunk_equals_prefill_rows_of_the_whole_sequence():
+    """A chunk continuing a sequence gives the rows of prefill over the whole
+    sequence at the chunk's positions (prefill is pinned to the brute-force
+    mask above)."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, d, t, n = 2, 4, 2, 8, 23, 9
+    spans = [1, 5, 40, 17]
+    k = rng.standard_normal((B, Hkv, t + n, d))
+    v = rng.standard_normal((B, Hkv, t + n, d))
+    q_full = rng.standard_normal((B, Hq, t + n, d))
+    want = attention.prefill(q_full, k, v, spans, 0.3)[:, :, t:, :]
+    got = attention.chunk(q_full[:, :, t:, :], [k[b] for b in range(B)], [v[b] for b in range(B)], [t, t], spans, 0.3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_chunk_at_position_zero_is_prefill_of_the_chunk():
+    rng = np.random.default_rng(32)
+    q = rng.standard_normal((1, 2, 11, 4))
+    k = rng.standard_normal((1, 1, 11, 4))
+    v = rng.standard_normal((1, 1, 11, 4))
+    got = attention.chunk(q, [k[0]], [v[0]], [0], [3, 11], 0.5)
+    np.testing.assert_allclose(got, attention.prefill(q, k, v, [3, 11], 0.5), rtol=0, atol=1e-12)
+
+
+def test_chunk_of_one_token_equals_ring_decode():
+    """n = 1 is one decode step: the ring-buffer emulation (its own pins in
+    test_oracle_kvcache) reads the same window through the ring."""
+    from oracle import kvcache as okv
+    rng = np.random.default_rng(33)
+    B, Hq, Hkv, d = 2, 4, 2, 8
+    spans = [7, 2, 12, 12]
+    caps = okv.group_capacities(spans, Hkv)
+    t = [30, 5]
+    hist_k = [rng.standard_normal((Hkv, tb + 1, d)) for tb in t]
+    hist_v = [rng.standard_normal((Hkv, tb + 1, d)) for tb in t]
+    q = rng.standard_normal((B, Hq, 1, d))
+    got = attention.chunk(q, hist_k, hist_v, t, spans, 0.25)[:, :, 0, :]
+    want = np.empty_like(got)
+    for b in range(B):
+        ring = okv.RingCache(1, Hkv, d, caps)
+        for p in range(t[b] + 1):
+            ring.append(hist_k[b][None, :, p:p + 1, :], hist_v[b][None, :, p:p + 1, :])
+        want[b] = okv.decode(ring, q[b:b + 1, :, 0, :], spans, 0.25)[0]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_chunk_rows_subset_and_shape_checks():
+    rng = np.random.default_rng(34)
+    q = rng.standard_normal((2, 2, 5, 4))
+    hk = [rng.standard_normal((1, 8, 4)), rng.standard_normal((1, 6, 4))]
+    hv = [rng.standard_normal((1, 8, 4)), rng.standard_normal((1, 6, 4))]
+    full = attention.chunk(q, hk, hv, [3, 1], [4, 2], 0.5)
+    rows = [(1, 0, 4), (0, 1, 0)]
+    np.testing.assert_array_equal(attention.chunk(q, hk, hv, [3, 1], [4, 2], 0.5, rows=rows),
+                                  np.stack([full[b, h, i] for b, h, i in rows]))
+    with pytest.raises(ValueError):
+        attention.chunk(q, hk, hv, [3, 2], [4, 2], 0.5)       # history length does not match t + n
