@@ -229,6 +229,44 @@ extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, v
   return launch_append(fill, k, v, (int32_t)N, s);
 }
 
+// Shared checks of the chunk entry points; MOA_OK when the call is well formed.
+static moa_status chunk_args(const moa_kv_cache* c, int32_t Hq, int32_t n, const int32_t* spans) {
+  if (!c || !spans) return MOA_ERR_INVALID_ARG;
+  if (Hq < 1 || Hq > MOA_MAX_HEADS || Hq % c->Hkv != 0 || n < 1) return MOA_ERR_INVALID_ARG;
+  const int32_t G = Hq / c->Hkv;
+  int32_t max_s = 1;
+  for (int32_t h = 0; h < Hq; ++h) {
+    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+    if (spans[h] > c->cap[h / G]) return MOA_ERR_CAPACITY;
+    max_s = std::max(max_s, spans[h]);
+  }
+  if ((int64_t)n + max_s + 128 > INT32_MAX) return MOA_ERR_INVALID_ARG;
+  if (c->dtype != MOA_BF16 || c->d != 128) return MOA_ERR_UNSUPPORTED;
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_chunk_workspace_bytes(const moa_kv_cache* c, int32_t Hq, int32_t n,
+                                                const int32_t* spans, size_t* bytes_out) {
+  if (!bytes_out) return MOA_ERR_INVALID_ARG;
+  const moa_status st = chunk_args(c, Hq, n, spans);
+  if (st != MOA_OK) return st;
+  *bytes_out = prefill_chunk_workspace_bytes(c->B, Hq, c->Hkv, n, spans);
+  return MOA_OK;
+}
+
+extern "C" moa_status moa_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, const void* v,
+                                        void* o, int32_t Hq, int32_t n, const int32_t* spans, float scale,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !o) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
+  const moa_status st = chunk_args(c, Hq, n, spans);
+  if (st != MOA_OK) return st;
+  if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
+  if (ws_bytes < prefill_chunk_workspace_bytes(c->B, Hq, c->Hkv, n, spans)) return MOA_ERR_WORKSPACE;
+  return launch_prefill_chunk(c, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
+}
+
 extern "C" moa_status moa_decode_append(moa_kv_cache* c, const void* q, const void* k, const void* v,
                                         void* o, int32_t Hq, const int32_t* spans, float scale, void* ws,
                                         size_t ws_bytes, void* stream) {

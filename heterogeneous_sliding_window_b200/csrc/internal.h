@@ -75,7 +75,8 @@ struct PrefillSchedule {
   std::vector<int32_t> off;     // n_ctas + 1
   std::vector<int32_t> units;   // 4 int32 per unit
 };
-PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas);
+PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
+                                 int32_t m0 = 0);
 // Rows (CTA, unit, b, h, query tile, first key tile, last key tile), one per query tile.
 std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, const int32_t* spans,
                                            int32_t n_ctas);
@@ -85,5 +86,17 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
                                int32_t B, int32_t Hq, int32_t Hkv, int32_t N,
                                const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                cudaStream_t s);
+
+// Chunked prefill (prefill_sm100.cu): the n new tokens of every sequence
+// attend to the cache's window plus themselves, then are appended.
+size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans);
+moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, const void* v, void* o,
+                                int32_t Hq, int32_t n, const int32_t* spans, float scale, void* ws,
+                                size_t ws_bytes, cudaStream_t s);
+// kv.cu: key/value rows of positions t_b - W .. t_b + n - 1 of every (b, g)
+// into sk, sv [B, Hkv, W + n, d]: the first W from the ring (zeros where the
+// position is negative or no longer held), the last n from the chunk k, v.
+moa_status launch_gather_window(const moa_kv_cache* c, const void* k, const void* v, int32_t n, int32_t W,
+                                void* sk, void* sv, cudaStream_t s);
 
 }  // namespace moa

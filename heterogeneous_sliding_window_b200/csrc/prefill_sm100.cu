@@ -102,7 +102,8 @@ constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
 constexpr uint32_t kUnitSlots = 4;                                // unit record ring depth
 constexpr uint32_t OFF_UNIT = (OFF_ABORT + 4 + 15) / 16 * 16;    // int4[kUnitSlots] unit records
-static_assert(OFF_UNIT + 16 * kUnitSlots <= OFF_BAR + 512, "barrier area");
+constexpr uint32_t OFF_KMIN = OFF_UNIT + 16 * kUnitSlots;         // int[kUnitSlots]: first valid key row
+static_assert(OFF_KMIN + 4 * kUnitSlots <= OFF_BAR + 512, "barrier area");
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 // Position in a ring of `n` stages: stage index and mbarrier phase parity.
@@ -118,7 +119,13 @@ struct PrefillParams {
   const int32_t* cta_off;        // units of CTA c: units[cta_off[c] .. cta_off[c+1])
   const int4* units;             // (b, h, m, loA), grouped by CTA, longest first within a CTA
   void* o;
-  int32_t N, Hq, Hkv, G;
+  // Key rows 0 .. N-1; query row r is key position q_off + r (q_off a
+  // multiple of 128), r < Nq.  A prompt has q_off = 0 and Nq = N.  A chunk
+  // continuing sequence b (t != nullptr) sees key rows below q_off - t[b] as
+  // positions before the sequence's start: they are masked.
+  int32_t N, Nq, q_off;
+  const int64_t* t;
+  int32_t Hq, Hkv, G;
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
 };
@@ -127,6 +134,7 @@ struct Ctx {
   uint32_t bar0;                       // address of barrier 0
   volatile int* abort;
   volatile int4* ring;                 // published unit records, kUnitSlots slots (x < 0: no more units)
+  volatile int* ring_kmin;             // per slot: the unit's first valid key row
   uint32_t* hdr;
   __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
   // Bounded wait that also gives up when another role has already failed.
@@ -160,16 +168,18 @@ struct Ctx {
   // Next unit record from the ring.  Single-thread roles (warp_wide = false)
   // release the slot themselves; warp-wide roles release it from lane 0 after
   // every lane has read it.
-  __device__ bool next_unit(uint32_t i, int lane, bool warp_wide, int4* u) const {
+  __device__ bool next_unit(uint32_t i, int lane, bool warp_wide, int4* u, int* kmin) const {
     const uint32_t slot = i % kUnitSlots, par = (i / kUnitSlots) & 1;
     if (warp_wide) {
       if (!wait_warp(B_UFULL0 + slot, par)) return false;
       *u = const_cast<const int4&>(ring[slot]);
+      *kmin = ring_kmin[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_UEMPTY0 + slot));
     } else {
       if (!wait(B_UFULL0 + slot, par)) return false;
       *u = const_cast<const int4&>(ring[slot]);
+      *kmin = ring_kmin[slot];
       mbar_arrive(bar(B_UEMPTY0 + slot));
     }
     return true;
@@ -183,23 +193,24 @@ __device__ __forceinline__ int first_key_tile(int t, int S) {
 
 // The unit's two query tiles: X = 0 (A, tile m) and X = 1 (B, tile m + 1).
 struct UnitInfo {
-  int S, zq, zk;
+  int S, zq, zk, kmin;
   int m[2], lo[2];
   bool hasB;
   int L, R;                            // shared key-tile range
   __device__ bool in(int X, int j) const { return (X == 0 || hasB) && j >= lo[X] && j <= m[X]; }
 };
 
-__device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const int4 U) {
+__device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const int4 U, int kmin) {
   UnitInfo x;
   x.S = p.span[U.y];
   x.zq = U.x * p.Hq + U.y;
   x.zk = U.x * p.Hkv + U.y / p.G;
+  x.kmin = kmin;
   x.m[0] = U.z;
-  x.lo[0] = U.w;
+  x.lo[0] = max(U.w, kmin >> 7);
   x.m[1] = U.z + 1;
   x.hasB = (long long)x.m[1] * 128 < (long long)p.N;
-  x.lo[1] = first_key_tile(x.m[1], x.S);
+  x.lo[1] = max(first_key_tile(x.m[1], x.S), kmin >> 7);
   x.L = x.lo[0];
   x.R = x.hasB ? x.m[1] : x.m[0];
   return x;
@@ -291,9 +302,10 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
   uint32_t tcount = 0, uc = 0;
   for (uint32_t i = 0;; ++i) {
     int4 U;
-    if (!c.next_unit(i, lane, true, &U)) return;
+    int kmin;
+    if (!c.next_unit(i, lane, true, &U, &kmin)) return;
     if (U.x < 0) return;
-    const UnitInfo x = decode_unit(p, U);
+    const UnitInfo x = decode_unit(p, U, kmin);
     if (X == 1 && !x.hasB) continue;
     const int i_row = x.m[X] * 128 + r;
     float m_run = -INFINITY, l_run = 0.f;            // m_run = -inf: no reference yet
@@ -301,7 +313,7 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
       if (!c.wait_warp(B_SFULL0 + X, tcount & 1)) return;
       tc_fence_after();
       const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
-      const int lo_c = i_row - x.S - kt * 128;       // keys c >  lo_c are inside the window
+      const int lo_c = max(i_row - x.S, x.kmin - 1) - kt * 128;   // keys c > lo_c are inside the window
       const bool edge = hi_c < 127 || lo_c >= 0;
       uint32_t w[64];                                // P of the tile, bf16 pairs
 #pragma unroll
@@ -367,9 +379,10 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
     }
     tc_fence_before();
     c.arrive_warp(B_OEMPTY0 + X);
-    if (i_row < p.N) {
+    const int o_row = i_row - p.q_off;
+    if (o_row < p.Nq) {
       uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                             ((size_t)x.zq * p.N + (size_t)i_row) * kD);
+                                             ((size_t)x.zq * p.Nq + (size_t)o_row) * kD);
 #pragma unroll
       for (int j = 0; j < 16; ++j) orow[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
     }
@@ -435,9 +448,10 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
   uint32_t tpA = 0, tpB = 0, ucA = 0, ucB = 0;       // PV tiles and units per stream
   uint32_t ui = 0;                                   // unit records read
   int4 U;
-  if (!c.next_unit(ui++, 0, false, &U)) return;
+  int kmin;
+  if (!c.next_unit(ui++, 0, false, &U, &kmin)) return;
   if (U.x < 0) return;
-  UnitInfo x = decode_unit(p, U);
+  UnitInfo x = decode_unit(p, U, kmin);
   QSlots q = take_q(x, nq);
   bool started_A = false;                            // S_A(L) of x already issued
   while (true) {
@@ -467,6 +481,7 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     // next unit, when its tile A could start during this unit's last step
     bool have_next = false, ended = false;
     int4 Uy = make_int4(0, 0, 0, 0);
+    int ykmin = 0;
     uint32_t ysA = 0, ypA = 0;
     for (int j = x.L; j <= x.R; ++j) {
       const bool more = j < x.R;
@@ -494,12 +509,12 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
         // Last step, tile B only: S_A of the next unit's first key tile (the
         // next K in the ring) goes to the tensor core now, so tile A's
         // softmax starts the next unit while tile B finishes this one.
-        if (!c.next_unit(ui++, 0, false, &Uy)) return;
+        if (!c.next_unit(ui++, 0, false, &Uy, &ykmin)) return;
         if (Uy.x < 0) {
           ended = true;
         } else {
-          // tile A of the next unit: query tile Uy.z, first key tile Uy.w; its
-          // Q slot is the next in the rotation
+          // tile A of the next unit: query tile Uy.z, first key tile
+          // max(Uy.w, ykmin / 128); its Q slot is the next in the rotation
           ysA = nq % kQSlots;
           ypA = (nq / kQSlots) & 1;
           if (!c.wait(B_KFULL0 + kst, kph)) return;
@@ -507,7 +522,7 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
           tc_fence_after();
           mma_qk(tSA, desc_qk_lo(sQ0 + ysA * kTileBytes), desc_qk_lo(sK0 + kst * kTileBytes), hi);
           mma_commit(c.bar(B_SFULL0));
-          if (Uy.w == Uy.z) mma_commit(c.bar(B_QEMPTY0 + ysA));
+          if (max(Uy.w, ykmin >> 7) == Uy.z) mma_commit(c.bar(B_QEMPTY0 + ysA));
           have_next = true;
         }
       }
@@ -545,14 +560,14 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     }
     if (ended) return;
     if (have_next) {
-      x = decode_unit(p, Uy);
+      x = decode_unit(p, Uy, ykmin);
       q = take_q(x, nq);                             // slot of tile A = ysA
       started_A = true;
       continue;
     }
-    if (!c.next_unit(ui++, 0, false, &U)) return;
+    if (!c.next_unit(ui++, 0, false, &U, &kmin)) return;
     if (U.x < 0) return;
-    x = decode_unit(p, U);
+    x = decode_unit(p, U, kmin);
     q = take_q(x, nq);
     started_A = false;
   }
@@ -573,8 +588,8 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
     if (!c.wait(B_QEMPTY0 + slot, par ^ 1)) return false;
     const uint32_t sQ = sQ0 + slot * kTileBytes;
     mbar_expect_tx(c.bar(B_QFULL0 + slot), kTileBytes);
-    tma_load_3d(sQ, tmQ, c.bar(B_QFULL0 + slot), 0, m * 128, zq);
-    tma_load_3d(sQ + kHalfBytes, tmQ, c.bar(B_QFULL0 + slot), 64, m * 128, zq);
+    tma_load_3d(sQ, tmQ, c.bar(B_QFULL0 + slot), 0, m * 128 - p.q_off, zq);
+    tma_load_3d(sQ + kHalfBytes, tmQ, c.bar(B_QFULL0 + slot), 64, m * 128 - p.q_off, zq);
     return true;
   };
   auto load_k = [&](int kt, int zk) -> bool {
@@ -597,9 +612,10 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
   };
   for (uint32_t i = 0;; ++i) {
     int4 U;
-    if (!c.next_unit(i, 0, false, &U)) return;
+    int kmin;
+    if (!c.next_unit(i, 0, false, &U, &kmin)) return;
     if (U.x < 0) return;
-    const UnitInfo x = decode_unit(p, U);
+    const UnitInfo x = decode_unit(p, U, kmin);
     // Loads in the MMA's order of use: Q_A, K(L), then per key tile j:
     // V(j), K(j+1); Q_B right before the first K tile that tile B uses.
     if (!load_q(x.m[0], x.zq)) return;
@@ -627,7 +643,13 @@ __device__ __forceinline__ void fetcher_role(const PrefillParams& p, const Ctx& 
     if (!c.wait(B_UEMPTY0 + slot, ((i / kUnitSlots) & 1) ^ 1)) return;
     const int u = first + (int)i;
     const int4 U = u < last ? p.units[u] : make_int4(-1, 0, 0, 0);
+    int kmin = 0;
+    if (p.t != nullptr && U.x >= 0) {
+      const long long f = (long long)p.q_off - p.t[U.x];
+      kmin = f > 0 ? (int)f : 0;
+    }
     const_cast<int4&>(c.ring[slot]) = U;
+    c.ring_kmin[slot] = kmin;
     mbar_arrive(c.bar(B_UFULL0 + slot));
     if (U.x < 0) return;
   }
@@ -648,6 +670,7 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   c.bar0 = sbase + OFF_BAR;
   c.abort = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   c.ring = reinterpret_cast<volatile int4*>(smem + OFF_UNIT);
+  c.ring_kmin = reinterpret_cast<volatile int*>(smem + OFF_KMIN);
   c.hdr = p.hdr;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM_SLOT);
 
@@ -739,14 +762,15 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 // longest first and dealt to n_ctas lists by the greedy longest-processing-
 // time rule (each unit to the list with the least work so far); a unit's work
 // is its (query tile, key tile) pairs plus a fixed per-unit overhead.
-PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas) {
-  const int64_t M = (N + kTileM - 1) / kTileM;      // query tiles
+PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
+                                 int32_t m0) {
+  const int64_t M = (N + kTileM - 1) / kTileM;      // key tiles; query tiles are m0 .. M-1
   struct U { int32_t b, h, m, lo; int64_t cost; };
   std::vector<U> v;
-  v.reserve((size_t)B * Hq * ((M + 1) / 2));
+  v.reserve((size_t)B * Hq * ((M - m0 + 1) / 2));
   for (int32_t b = 0; b < B; ++b)
     for (int32_t h = 0; h < Hq; ++h)
-      for (int64_t m = 0; m < M; m += 2) {
+      for (int64_t m = m0; m < M; m += 2) {
         const int64_t lo = first_tile_host(m, spans[h]);
         int64_t cost = m - lo + 1 + kUnitOverheadTiles;
         if (m + 1 < M) cost += m + 1 - first_tile_host(m + 1, spans[h]) + 1;
@@ -805,22 +829,29 @@ size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
   return kUnitsOffset + (size_t)B * Hq * M * 16;
 }
 
-moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
-                               int32_t Hq, int32_t Hkv, int32_t N, const int32_t* spans, float scale,
-                               void* ws, size_t ws_bytes, cudaStream_t s) {
-  if (ws_bytes < prefill_workspace_bytes(B, Hq, N)) return MOA_ERR_WORKSPACE;
+namespace {
+
+// Query rows 0 .. Nq-1 are key positions q_off .. q_off+Nq-1 of key rows
+// 0 .. Nk-1 (q_off a multiple of 128); t: per-sequence token counts of a
+// chunk (rows below q_off - t[b] masked), or nullptr for a prompt.
+moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, void* o, int32_t B,
+                                    int32_t Hq, int32_t Hkv, int32_t Nq, int32_t Nk, int32_t q_off,
+                                    const int64_t* t, const int32_t* spans, float scale, void* ws,
+                                    size_t ws_bytes, cudaStream_t s) {
+  if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, N, (int64_t)B * Hq) || !make_map(&mk, k, N, (int64_t)B * Hkv) ||
-      !make_map(&mv, v, N, (int64_t)B * Hkv))
+  if (!make_map(&mq, q, Nq, (int64_t)B * Hq) || !make_map(&mk, k, Nk, (int64_t)B * Hkv) ||
+      !make_map(&mv, v, Nk, (int64_t)B * Hkv))
     return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
   // Header (error word, zeroed), the per-CTA list offsets and the units,
   // uploaded in one copy.  The pageable source is staged by the runtime
   // before cudaMemcpyAsync returns.
-  const int64_t M = (N + kTileM - 1) / kTileM;
-  const int64_t n_units = (int64_t)B * Hq * ((M + 1) / 2);
+  const int32_t m0 = q_off / kTileM;
+  const int64_t Mq = (Nq + kTileM - 1) / kTileM;
+  const int64_t n_units = (int64_t)B * Hq * ((Mq + 1) / 2);
   const int32_t grid = (int32_t)std::min<int64_t>({n_units, (int64_t)sm_count(), (int64_t)kPrefillMaxCtas});
-  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, grid);
+  const PrefillSchedule sch = prefill_schedule(B, Hq, Nk, spans, grid, m0);
   std::vector<int32_t> blob(kUnitsOffset / 4 + sch.units.size(), 0);
   std::copy(sch.off.begin(), sch.off.end(), blob.begin() + kOffsOffset / 4);
   std::copy(sch.units.begin(), sch.units.end(), blob.begin() + kUnitsOffset / 4);
@@ -832,7 +863,10 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
   p.cta_off = reinterpret_cast<const int32_t*>((char*)ws + kOffsOffset);
   p.units = reinterpret_cast<const int4*>((char*)ws + kUnitsOffset);
   p.o = o;
-  p.N = N;
+  p.N = Nk;
+  p.Nq = Nq;
+  p.q_off = q_off;
+  p.t = t;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -848,6 +882,54 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "prefill smem attribute");
   prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, p);
   return check_launch("prefill_bf16 launch");
+}
+
+// Chunk workspace: the prefill schedule region, then the gathered key and
+// value rows [B, Hkv, W + n, d] (W = prior keys any query can reach,
+// rounded up to a tile).
+struct ChunkLayout {
+  int32_t W = 0, Nk = 0;
+  size_t off_k = 0, off_v = 0, bytes = 0;
+};
+
+ChunkLayout chunk_layout(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans) {
+  ChunkLayout L;
+  int32_t max_s = 1;
+  for (int h = 0; h < Hq; ++h) max_s = std::max(max_s, spans[h]);
+  L.W = (max_s - 1 + kTileN - 1) / kTileN * kTileN;
+  L.Nk = L.W + n;
+  const size_t rows = (size_t)B * Hkv * (size_t)L.Nk * kD * 2;
+  L.off_k = (prefill_workspace_bytes(B, Hq, n) + 255) / 256 * 256;
+  L.off_v = L.off_k + (rows + 255) / 256 * 256;
+  L.bytes = L.off_v + rows;
+  return L;
+}
+
+}  // namespace
+
+moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
+                               int32_t Hq, int32_t Hkv, int32_t N, const int32_t* spans, float scale,
+                               void* ws, size_t ws_bytes, cudaStream_t s) {
+  return launch_prefill_bf16_rows(q, k, v, o, B, Hq, Hkv, N, N, 0, nullptr, spans, scale, ws, ws_bytes, s);
+}
+
+size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans) {
+  return chunk_layout(B, Hq, Hkv, n, spans).bytes;
+}
+
+moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, const void* v, void* o,
+                                int32_t Hq, int32_t n, const int32_t* spans, float scale, void* ws,
+                                size_t ws_bytes, cudaStream_t s) {
+  const ChunkLayout L = chunk_layout(c->B, Hq, c->Hkv, n, spans);
+  if (ws_bytes < L.bytes) return MOA_ERR_WORKSPACE;
+  char* sk = static_cast<char*>(ws) + L.off_k;
+  char* sv = static_cast<char*>(ws) + L.off_v;
+  moa_status st = launch_gather_window(c, k, v, n, L.W, sk, sv, s);
+  if (st != MOA_OK) return st;
+  const int64_t* t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
+  st = launch_prefill_bf16_rows(q, sk, sv, o, c->B, Hq, c->Hkv, n, L.Nk, L.W, t, spans, scale, ws, L.off_k, s);
+  if (st != MOA_OK) return st;
+  return launch_append(c, k, v, n, s);
 }
 
 }  // namespace moa

@@ -24,7 +24,8 @@ EXPORTS = (
     "moa_status_string", "moa_rules_eval", "moa_kv_bytes", "moa_kv_header_bytes", "moa_kv_alloc",
     "moa_kv_free", "moa_kv_append", "moa_kv_positions", "moa_kv_set_positions", "moa_kv_layout",
     "moa_workspace_bytes", "moa_workspace_init", "moa_workspace_check", "moa_prefill",
-    "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws", "moa_stream_read",
+    "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws", "moa_stream_read", "moa_chunk_workspace_bytes",
+    "moa_prefill_chunk",
 )
 
 
@@ -68,6 +69,8 @@ def load():
         "moa_decode_append": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_static_ws": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp]),
         "moa_stream_read": (ctypes.c_int, [vp, sz, vp, vp]),
+        "moa_chunk_workspace_bytes": (ctypes.c_int, [vp, i32, i32, P(i32), P(sz)]),
+        "moa_prefill_chunk": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, P(i32), f32, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -235,6 +238,20 @@ def moa_decode_static_ws(handle, q, o, Hq, spans, scale, stream=None):
     sp, spp = _i32(spans)
     _check(load().moa_decode_static_ws(handle, _ptr(q), _ptr(o), Hq, spp, float(scale), _stream(stream)),
            "moa_decode_static_ws")
+
+
+def moa_chunk_workspace_bytes(handle, Hq, n, spans):
+    sp, spp = _i32(spans)
+    out = ctypes.c_size_t(0)
+    _check(load().moa_chunk_workspace_bytes(handle, Hq, n, spp, ctypes.byref(out)), "moa_chunk_workspace_bytes")
+    return out.value
+
+
+def moa_prefill_chunk(handle, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, stream=None):
+    """The n new tokens of every sequence attend to the cache's window and themselves, then are appended."""
+    sp, spp = _i32(spans)
+    _check(load().moa_prefill_chunk(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), Hq, n, spp, float(scale),
+                                    _ptr(ws), int(ws_bytes), _stream(stream)), "moa_prefill_chunk")
 
 
 def moa_stream_read(buf, nbytes, out, stream=None):

@@ -196,6 +196,32 @@ moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t*
                                 int64_t* n_rows_out);
 
 /* ---------------------------------------------------------------------------
+ * Chunked prefill: a prompt that arrives in pieces, served from the same
+ * fixed-size per-head cache as decode ("Mixture of Attention" project page,
+ * "Demo" step 03; the windowed attention of "Finding two" at an offset).
+ * Sequence b holds t_b tokens in `cache`; q, k, v hold its next n tokens
+ * (positions t_b .. t_b+n-1).  Query i of head h attends to positions
+ * j in (t_b + i - S_h, t_b + i], j >= 0: the older ones read through the
+ * ring, the chunk's own from k, v.  Then the chunk is appended (the cache
+ * ends as after moa_kv_append(cache, k, v, n)).  With t_b = 0 this is
+ * moa_prefill of the chunk with fill.
+ *   q, o: device [B, Hq, n, d]; k, v: device [B, Hkv, n, d]; all 16-byte
+ *   aligned, bf16, d = 128 (other caches: MOA_ERR_UNSUPPORTED).
+ *   spans: host int32[Hq], 1 <= spans[h] <= C_{h/(Hq/Hkv)}, else
+ *   MOA_ERR_CAPACITY.
+ *   workspace: moa_chunk_workspace_bytes(...) bytes, 256-byte aligned, no
+ *   initialisation needed; it holds the work-unit schedule and the gathered
+ *   key/value rows [B, Hkv, W + n, d], W = max_h S_h - 1 rounded up to 128.
+ * Three launches on `stream`: the window gather, the tensor-core prefill
+ * kernel (query rows offset by W into the gathered rows, rows of negative
+ * positions masked), the append.  Errors as moa_prefill. */
+moa_status moa_chunk_workspace_bytes(const moa_kv_cache* cache, int32_t Hq, int32_t n,
+                                     const int32_t* spans, size_t* bytes_out);
+moa_status moa_prefill_chunk(moa_kv_cache* cache, const void* q, const void* k, const void* v,
+                             void* o, int32_t Hq, int32_t n, const int32_t* spans, float scale,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Decode: one new query token per sequence against the ring cache.  Call
  * moa_kv_append for the token's k, v first; then query head h of sequence b
  * (at position t_b - 1) attends to positions j in (t_b - 1 - S_h, t_b - 1],

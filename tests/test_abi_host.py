@@ -191,6 +191,18 @@ def test_stream_read_argument_errors_need_no_gpu():
         assert e.value.status == moa.MOA_ERR_INVALID_ARG, (buf, nbytes, out)
 
 
+def test_prefill_chunk_argument_errors_need_no_gpu():
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_chunk_workspace_bytes(None, 4, 128, [64] * 4)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_prefill_chunk(None, 4096, 4096, 4096, 4096, 4, 128, [64] * 4, 0.088, 4096, 1 << 20, 0)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    with pytest.raises(moa.MoaError) as e:      # misaligned q is rejected before the cache is looked at
+        moa.moa_prefill_chunk(None, 4100, 4096, 4096, 4096, 4, 128, [64] * 4, 0.088, 4096, 1 << 20, 0)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes():
     spans = [64, 300, 4096, 1]
     d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)

@@ -483,3 +483,166 @@ def test_stream_read_checksum(nbytes):
     hi = int(np.bitwise_xor.reduce(host[0::2])) if nbytes else 0
     lo = int(np.bitwise_xor.reduce(host[1::2])) if nbytes else 0
     assert got == (hi << 32) | lo
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill: pieces of a prompt attend to the ring's window and to
+# themselves, then are appended
+# ---------------------------------------------------------------------------
+def _chunk_call(cache, q, k, v, Hq, spans, scale):
+    B, _, n, d = q.shape
+    nb = moa.moa_chunk_workspace_bytes(cache.handle, Hq, n, spans)
+    buf = torch.empty(nb + 256, dtype=torch.uint8, device=DEV)
+    ptr = (buf.data_ptr() + 255) // 256 * 256
+    o = _nan_like((B, Hq, n, d), torch.bfloat16)
+    moa.moa_prefill_chunk(cache.handle, q, k, v, o, Hq, n, spans, scale, ptr, nb)
+    torch.cuda.synchronize()
+    return o
+
+
+CHUNK_CASES = [
+    # (B, Hq, Hkv, spans, chunk sizes in order)
+    (2, 4, 2, [300, 64, 129, 1], [500, 200, 77]),                # first chunk into an empty cache
+    (1, 2, 1, [40, 700], [128, 1, 300, 256, 129]),               # tile-aligned, one token, ragged
+    (3, 8, 2, [40, 38, 64, 64, 300, 299, 299, 280], [257, 130]),  # GQA, 4 query heads per kv head
+    (1, 4, 4, [1, 2, 3, 1000], [700, 700]),                      # ring wraps inside a chunk
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_CASES, ids=lambda c: "B%d_H%d_%d_%s" % (c[0], c[1], c[2],
+                                                                            "-".join(map(str, c[4]))))
+def test_bf16_prefill_chunks_match_oracle(case):
+    B, Hq, Hkv, spans, pieces = case
+    d = 128
+    scale = 1.0 / math.sqrt(d)
+    T = sum(pieces)
+    q = inputs.randn(80, (B, Hq, T, d))
+    k = inputs.randn(81, (B, Hkv, T, d))
+    v = inputs.randn(82, (B, Hkv, T, d))
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    qf, kf, vf = inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v)
+    t = 0
+    for n in pieces:
+        sl = slice(t, t + n)
+        o = _chunk_call(cache, q[:, :, sl].contiguous().to(DEV), k[:, :, sl].contiguous().to(DEV),
+                        v[:, :, sl].contiguous().to(DEV), Hq, spans, scale)
+        want = oatt.chunk(qf[:, :, sl], [kf[b, :, :t + n] for b in range(B)], [vf[b, :, :t + n] for b in range(B)],
+                          [t] * B, spans, scale)
+        err = np.max(np.abs(inputs.as_f64(o) - want))
+        assert err <= BF16_TOL, (t, n, err)
+        ring.append(kf[:, :, sl], vf[:, :, sl])
+        t += n
+        assert cache.positions() == [t] * B
+        assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "bf16")
+
+
+def test_bf16_prefill_chunk_with_a_different_history_per_sequence():
+    """Sequences at different positions (one shorter than every window, one
+    empty): rows of negative positions are masked per sequence."""
+    B, Hq, Hkv, d = 3, 4, 2, 128
+    spans = [333, 64, 700, 5]
+    scale = 1.0 / math.sqrt(d)
+    t = [1000, 37, 0]
+    n = 190
+    caps = okv.group_capacities(spans, Hkv)
+    hist_k = [inputs.randn(90 + b, (1, Hkv, t[b] + n, d)) for b in range(B)]
+    hist_v = [inputs.randn(95 + b, (1, Hkv, t[b] + n, d)) for b in range(B)]
+    image = b""
+    for b in range(B):
+        ring = okv.RingCache(1, Hkv, d, caps)
+        if t[b]:
+            ring.append(inputs.as_f64(hist_k[b][:, :, :t[b]]), inputs.as_f64(hist_v[b][:, :, :t[b]]))
+        image += okv.data_image(ring, "bf16")
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    cache.data_bytes().copy_(torch.frombuffer(bytearray(image), dtype=torch.uint8).to(DEV))
+    cache.set_positions(t)
+    q = inputs.randn(99, (B, Hq, n, d))
+    kc = torch.cat([hist_k[b][:, :, t[b]:] for b in range(B)], dim=0)
+    vc = torch.cat([hist_v[b][:, :, t[b]:] for b in range(B)], dim=0)
+    o = _chunk_call(cache, q.to(DEV), kc.contiguous().to(DEV), vc.contiguous().to(DEV), Hq, spans, scale)
+    want = oatt.chunk(inputs.as_f64(q), [inputs.as_f64(hist_k[b])[0] for b in range(B)],
+                      [inputs.as_f64(hist_v[b])[0] for b in range(B)], t, spans, scale)
+    assert np.max(np.abs(inputs.as_f64(o) - want)) <= BF16_TOL
+    assert cache.positions() == [tb + n for tb in t]
+
+
+def test_bf16_prefill_chunk_then_decode():
+    """Decode after a chunked prompt reads the cache the chunks left."""
+    B, Hq, Hkv, d = 2, 4, 2, 128
+    spans = [257, 64, 500, 3]
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    t = 0
+    for i, n in enumerate([300, 211]):
+        q = inputs.randn(110 + i, (B, Hq, n, d))
+        k = inputs.randn(120 + i, (B, Hkv, n, d))
+        v = inputs.randn(130 + i, (B, Hkv, n, d))
+        _chunk_call(cache, q.to(DEV), k.to(DEV), v.to(DEV), Hq, spans, scale)
+        ring.append(inputs.as_f64(k), inputs.as_f64(v))
+        t += n
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    qd = inputs.randn(140, (B, Hq, d))
+    kd = inputs.randn(141, (B, Hkv, 1, d))
+    vd = inputs.randn(142, (B, Hkv, 1, d))
+    o = _nan_like((B, Hq, d), torch.bfloat16)
+    moa.moa_decode_append(cache.handle, qd.to(DEV), kd.to(DEV), vd.to(DEV), o, Hq, spans, scale, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    ring.append(inputs.as_f64(kd), inputs.as_f64(vd))
+    want = okv.decode(ring, inputs.as_f64(qd), spans, scale)
+    assert np.max(np.abs(inputs.as_f64(o) - want)) <= BF16_TOL
+
+
+def test_bf16_prefill_chunk_vicuna7b_shaped_sampled():
+    """A 1024-token chunk after a 4096-token prompt, 32 heads at 25 % density:
+    sampled rows against the oracle, the rest checked finite."""
+    B, H, d, t, n = 1, 32, 128, 4096, 1024
+    pa, pb = inputs.tables_7b(5, H, t + n, 64, 0.25, orules.eval_spans)
+    spans = [int(s) for s in orules.eval_spans(pa, pb, t + n, 64)]
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(150, (B, H, t + n, d))
+    k = inputs.randn_cuda(151, (B, H, t + n, d))
+    v = inputs.randn_cuda(152, (B, H, t + n, d))
+    caps = okv.group_capacities(spans, H)
+    cache = moa.KVCache(B, H, d, "bf16", caps)
+    _chunk_call(cache, q[:, :, :t].contiguous(), k[:, :, :t].contiguous(), v[:, :, :t].contiguous(), H, spans, scale)
+    o = _chunk_call(cache, q[:, :, t:].contiguous(), k[:, :, t:].contiguous(), v[:, :, t:].contiguous(), H, spans,
+                    scale)
+    assert torch.isfinite(o.float()).all()
+    rng = np.random.default_rng(3)
+    rows = [(0, int(h), int(i)) for h, i in zip(rng.integers(0, H, 48), rng.integers(0, n, 48))]
+    rows += [(0, 0, 0), (0, H - 1, n - 1)]
+    kf = inputs.as_f64(k)
+    vf = inputs.as_f64(v)
+    want = oatt.chunk(inputs.as_f64(q[:, :, t:]), [kf[0]], [vf[0]], [t], spans, scale, rows=rows)
+    got = inputs.as_f64(o)
+    err = max(np.max(np.abs(got[b, h, i] - want[r])) for r, (b, h, i) in enumerate(rows))
+    assert err <= BF16_TOL
+    assert cache.positions() == [t + n]
+
+
+def test_prefill_chunk_errors():
+    cache = moa.KVCache(1, 2, 128, "bf16", [64, 64])
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_chunk_workspace_bytes(cache.handle, 4, 10, [65, 1, 1, 1])
+    assert e.value.status == moa.MOA_ERR_CAPACITY
+    f32 = moa.KVCache(1, 1, 64, "f32", [8])
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_chunk_workspace_bytes(f32.handle, 1, 10, [8])
+    assert e.value.status == moa.MOA_ERR_UNSUPPORTED
+    spans = [64, 1, 1, 1]
+    nb = moa.moa_chunk_workspace_bytes(cache.handle, 4, 10, spans)
+    buf = torch.empty(nb + 256, dtype=torch.uint8, device=DEV)
+    ptr = (buf.data_ptr() + 255) // 256 * 256
+    q = torch.zeros((1, 4, 10, 128), dtype=torch.bfloat16, device=DEV)
+    kv = torch.zeros((1, 2, 10, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_prefill_chunk(cache.handle, q, kv, kv, q.clone(), 4, 10, spans, 0.088, ptr, nb - 1)
+    assert e.value.status == moa.MOA_ERR_WORKSPACE
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_prefill_chunk(cache.handle, q, kv, kv, q.clone(), 4, 0, spans, 0.088, ptr, nb)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    assert cache.positions() == [0]
