@@ -370,6 +370,7 @@ def run_ours(args):
     h2d = sum(x.numel() * x.element_size() for x in h_q + h_k + h_v)
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
+    chunk = chunk_prefill(stream, tf_peak, peak_kind)
     read_gbs = read_only_gbs([c.data_bytes() for c in caches[:4]], stream)
 
     result = None
@@ -407,6 +408,7 @@ def run_ours(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "note": "decode step through the C ABI from pinned host q/k/v to host o"},
             "gqa_decode": gqa,
+            "prefill_chunk": chunk,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clock_info,
             "cpu_baseline": {"value": round(cpu_tok, 4), "unit": "tokens/s", "cores": _oracle_threads(),
@@ -440,6 +442,53 @@ def read_only_gbs(bufs, stream, reps=5):
         torch.cuda.synchronize()
         best = min(best, e0.elapsed_time(e1))
     return sum(sizes) / (best * 1e-3) / 1e9
+
+
+def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
+    """Chunked prefill into the ring cache: a Vicuna-7B-shaped layer (32 heads,
+    d=128, spans at 25 % of 8192) holds the first 4096 tokens of a prompt and
+    takes the other 4096 in one moa_prefill_chunk call (window gather,
+    attention, append).
+    In-window TFLOP/s of the chunk's rows over the call's device time; the
+    positions are reset between calls, outside the timed events."""
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    B, H, d, t, n = 1, 32, 128, 4096, 4096
+    a, b = inputs.tables_7b(P_SEED + 1, H, t + n, BLOCK, P_DENSITY, moa.moa_rules_eval)
+    spans = moa.moa_rules_eval(a, b, t + n, BLOCK)
+    scale = 1.0 / math.sqrt(d)
+    cache = moa.KVCache(B, H, d, "bf16", spans)
+    nb = max(moa.moa_chunk_workspace_bytes(cache.handle, H, t, spans),
+             moa.moa_chunk_workspace_bytes(cache.handle, H, n, spans))
+    wbuf = torch.empty(nb + 256, dtype=torch.uint8, device="cuda")
+    wptr = (wbuf.data_ptr() + 255) // 256 * 256
+    q = inputs.randn_cuda(500, (B, H, t + n, d))
+    k = inputs.randn_cuda(501, (B, H, t + n, d))
+    v = inputs.randn_cuda(502, (B, H, t + n, d))
+    q0, k0, v0 = q[:, :, :t].contiguous(), k[:, :, :t].contiguous(), v[:, :, :t].contiguous()
+    q1, k1, v1 = q[:, :, t:].contiguous(), k[:, :, t:].contiguous(), v[:, :, t:].contiguous()
+    o0 = torch.empty_like(q0)
+    o1 = torch.empty_like(q1)
+    moa.moa_prefill_chunk(cache.handle, q0, k0, v0, o0, H, t, spans, scale, wptr, nb, stream)
+    flops = sum(4 * d * sum(min(t + i + 1, S) for i in range(n)) for S in spans) * B
+    times = []
+    for r in range(reps + 3):
+        cache.set_positions([t], stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moa.moa_prefill_chunk(cache.handle, q1, k1, v1, o1, H, n, spans, scale, wptr, nb, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if r >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": "vicuna7b-shaped layer: 4096-token chunk after 4096 cached tokens, H=32 d=128, "
+                        "spans at 25% of 8192",
+            "ms": round(ms, 4), "in_window_flops": int(flops), "tflops": round(tf, 2),
+            "frac": round(tf / tf_peak, 4), "peak_kind": peak_kind + " burst (bf16_tflops)",
+            "launches": 3}
 
 
 def gqa_decode_layer(stream, reps=20):
@@ -540,6 +589,8 @@ def run_profile_case(case, launches=3):
 
     prefill: the 7B prompt (B=1, 32 heads, N=8192; Q/K/V 192 MiB), `launches` prefills.
     decode : one decode layer of the 7B workload (B=32, 32 heads, context 4096; 1 GiB cache).
+    chunk  : the bench's chunked prefill (4096-token chunk after 4096 cached tokens, 32 heads),
+             `launches` calls of moa_prefill_chunk (gather, prefill kernel, append each).
     """
     import torch
     from heterogeneous_sliding_window_b200 import inputs, moa
@@ -556,6 +607,23 @@ def run_profile_case(case, launches=3):
             moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", sp, 1.0 / math.sqrt(P_D), ws.ptr,
                             ws.nbytes)
         moa.moa_workspace_check(ws.ptr)
+    elif case == "chunk":
+        H, d, t, n = 32, 128, 4096, 4096
+        a, b = inputs.tables_7b(P_SEED + 1, H, t + n, BLOCK, P_DENSITY, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, t + n, BLOCK)
+        c = moa.KVCache(1, H, d, "bf16", sp)
+        nb = max(moa.moa_chunk_workspace_bytes(c.handle, H, t, sp), moa.moa_chunk_workspace_bytes(c.handle, H, n, sp))
+        wbuf = torch.empty(nb + 256, dtype=torch.uint8, device="cuda")
+        wptr = (wbuf.data_ptr() + 255) // 256 * 256
+        q = inputs.randn_cuda(500, (1, H, t, d))
+        k = inputs.randn_cuda(501, (1, H, t, d))
+        v = inputs.randn_cuda(502, (1, H, t, d))
+        o = torch.empty_like(q)
+        moa.moa_prefill_chunk(c.handle, q, k, v, o, H, t, sp, 1.0 / math.sqrt(d), wptr, nb)
+        for _ in range(launches):
+            c.set_positions([t])
+            moa.moa_prefill_chunk(c.handle, q, k, v, o, H, n, sp, 1.0 / math.sqrt(d), wptr, nb)
+        c.positions()
     else:
         a, b = inputs.tables_7b(D_SEED, D_H, D_N, BLOCK, D_DENSITY, moa.moa_rules_eval)
         sp = moa.moa_rules_eval(a, b, D_N, BLOCK)
@@ -577,7 +645,7 @@ def run_profile_case(case, launches=3):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "chunk"], default=None,
                     help="run one small single-kernel case (for ncu) and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)

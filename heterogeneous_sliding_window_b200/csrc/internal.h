@@ -93,10 +93,10 @@ size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t
 moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, const void* v, void* o,
                                 int32_t Hq, int32_t n, const int32_t* spans, float scale, void* ws,
                                 size_t ws_bytes, cudaStream_t s);
-// kv.cu: key/value rows of positions t_b - W .. t_b + n - 1 of every (b, g)
-// into sk, sv [B, Hkv, W + n, d]: the first W from the ring (zeros where the
-// position is negative or no longer held), the last n from the chunk k, v.
-moa_status launch_gather_window(const moa_kv_cache* c, const void* k, const void* v, int32_t n, int32_t W,
-                                void* sk, void* sv, cudaStream_t s);
+// kv.cu: key/value rows of positions t_b - W .. t_b - 1 of every (b, g) into
+// sk, sv [B, Hkv, W, d], read through the ring (zeros where the position is
+// negative or no longer held).  Only rows W - C_g + 1 - 127 and up, rounded
+// down to a tile, are written: no query of the group's heads reaches below.
+moa_status launch_gather_window(const moa_kv_cache* c, int32_t W, void* sk, void* sv, cudaStream_t s);
 
 }  // namespace moa

@@ -4,6 +4,8 @@
 // from a fixed-size KV cache sized per head.  Token position p of a sequence
 // is kept in slot p mod C_g of its key/value head g, so the buffer always
 // holds the last C_g tokens -- all that a head with span S_h <= C_g reads.
+#include <algorithm>
+
 #include "internal.h"
 
 namespace moa {
@@ -67,19 +69,19 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const __grid_con
   }
 }
 
-// Window gather for a chunk: rows r < W of (b, g) are positions t_b - W + r
-// read through the ring (zeros for positions below 0 or older than the ring
-// holds), rows W .. W+n-1 are the chunk's own keys and values.
+// Window gather for a chunk: row r of (b, g) is position t_b - W + r, read
+// through the ring (zeros for positions below 0 or older than the ring
+// holds).  Rows below R_g = 128 * floor((W - C_g + 1) / 128) are never in a
+// visited key tile of the group's heads (every span is <= C_g), so they are
+// skipped.
 constexpr int kGatherRows = 64;
 
 struct GatherParams {
   const char* data;           // data region of the cache buffer
   const int64_t* t;           // header: tokens per sequence
-  const char* k;              // chunk [B, Hkv, n, d]
-  const char* v;
-  char* sk;                   // [B, Hkv, W + n, d]
+  char* sk;                   // [B, Hkv, W, d]
   char* sv;
-  int32_t Hkv, n, W, row_bytes;
+  int32_t Hkv, W, row_bytes;
   int64_t sumC;
   int32_t cap[MOA_MAX_HEADS];
   int64_t goff[MOA_MAX_HEADS];
@@ -89,31 +91,25 @@ __global__ void __launch_bounds__(kAppendThreads) gather_window_kernel(const __g
   const int g = blockIdx.y;
   const int b = blockIdx.z;
   const int C = p.cap[g];
-  const int rows_total = p.W + p.n;
-  const int r0 = blockIdx.x * kGatherRows;
-  if (r0 >= rows_total) return;
-  const int rows = min(kGatherRows, rows_total - r0);
+  const int lowest = p.W - C + 1 > 0 ? (p.W - C + 1) / 128 * 128 : 0;
+  const int r0 = lowest + blockIdx.x * kGatherRows;
+  if (r0 >= p.W) return;
+  const int rows = min(kGatherRows, p.W - r0);
   const int vpr = p.row_bytes / 16;
   const int64_t t0 = p.t[b];
   const char* kring = p.data + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * p.row_bytes;
   const char* vring = kring + (size_t)C * p.row_bytes;
-  const size_t zrow = ((size_t)b * p.Hkv + g) * (size_t)rows_total;
+  const size_t zrow = ((size_t)b * p.Hkv + g) * (size_t)p.W;
   for (int idx = threadIdx.x; idx < rows * vpr; idx += kAppendThreads) {
     const int rr = idx / vpr;
     const int vv = idx - rr * vpr;
     const int r = r0 + rr;
     int4 kx = make_int4(0, 0, 0, 0), vx = make_int4(0, 0, 0, 0);
-    if (r < p.W) {
-      const int64_t pos = t0 - p.W + r;
-      if (pos >= 0 && pos >= t0 - C) {
-        const size_t src = (size_t)(pos % C) * p.row_bytes + (size_t)vv * 16;
-        kx = __ldg(reinterpret_cast<const int4*>(kring + src));
-        vx = __ldg(reinterpret_cast<const int4*>(vring + src));
-      }
-    } else {
-      const size_t src = (((size_t)b * p.Hkv + g) * (size_t)p.n + (r - p.W)) * p.row_bytes + (size_t)vv * 16;
-      kx = __ldg(reinterpret_cast<const int4*>(p.k + src));
-      vx = __ldg(reinterpret_cast<const int4*>(p.v + src));
+    const int64_t pos = t0 - p.W + r;
+    if (pos >= 0 && pos >= t0 - C) {
+      const size_t src = (size_t)(pos % C) * p.row_bytes + (size_t)vv * 16;
+      kx = __ldg(reinterpret_cast<const int4*>(kring + src));
+      vx = __ldg(reinterpret_cast<const int4*>(vring + src));
     }
     const size_t dst = (zrow + r) * p.row_bytes + (size_t)vv * 16;
     *reinterpret_cast<int4*>(p.sk + dst) = kx;
@@ -123,25 +119,24 @@ __global__ void __launch_bounds__(kAppendThreads) gather_window_kernel(const __g
 
 }  // namespace
 
-moa_status launch_gather_window(const moa_kv_cache* c, const void* k, const void* v, int32_t n, int32_t W,
-                                void* sk, void* sv, cudaStream_t s) {
+moa_status launch_gather_window(const moa_kv_cache* c, int32_t W, void* sk, void* sv, cudaStream_t s) {
   GatherParams p;
   p.data = c->buf + c->header;
   p.t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
-  p.k = (const char*)k;
-  p.v = (const char*)v;
   p.sk = (char*)sk;
   p.sv = (char*)sv;
   p.Hkv = c->Hkv;
-  p.n = n;
   p.W = W;
   p.row_bytes = c->d * (int)elem_bytes(c->dtype);
   p.sumC = c->goff[c->Hkv];
+  int max_rows = 0;
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
     p.goff[g] = c->goff[g];
+    const int lowest = W - c->cap[g] + 1 > 0 ? (W - c->cap[g] + 1) / 128 * 128 : 0;
+    max_rows = std::max(max_rows, W - lowest);
   }
-  dim3 grid((W + n + kGatherRows - 1) / kGatherRows, c->Hkv, c->B);
+  dim3 grid((max_rows + kGatherRows - 1) / kGatherRows, c->Hkv, c->B);
   gather_window_kernel<<<grid, kAppendThreads, 0, s>>>(p);
   return check_launch("window gather launch");
 }

@@ -122,7 +122,9 @@ struct PrefillParams {
   // Key rows 0 .. N-1; query row r is key position q_off + r (q_off a
   // multiple of 128), r < Nq.  A prompt has q_off = 0 and Nq = N.  A chunk
   // continuing sequence b (t != nullptr) sees key rows below q_off - t[b] as
-  // positions before the sequence's start: they are masked.
+  // positions before the sequence's start: they are masked.  Key rows below
+  // q_off come from the window maps, rows q_off.. from the K/V maps at row
+  // (key row - q_off).
   int32_t N, Nq, q_off;
   const int64_t* t;
   int32_t Hq, Hkv, G;
@@ -307,9 +309,13 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
     if (U.x < 0) return;
     const UnitInfo x = decode_unit(p, U, kmin);
     if (X == 1 && !x.hasB) continue;
-    const int i_row = x.m[X] * 128 + r;
+    // this warpgroup's query tile and first key tile, selected rather than
+    // indexed so the unit record stays in registers
+    const int m_x = X ? x.m[1] : x.m[0];
+    const int lo_x = X ? x.lo[1] : x.lo[0];
+    const int i_row = m_x * 128 + r;
     float m_run = -INFINITY, l_run = 0.f;            // m_run = -inf: no reference yet
-    for (int kt = x.lo[X]; kt <= x.m[X]; ++kt, ++tcount) {
+    for (int kt = lo_x; kt <= m_x; ++kt, ++tcount) {
       if (!c.wait_warp(B_SFULL0 + X, tcount & 1)) return;
       tc_fence_after();
       const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
@@ -333,7 +339,7 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
             m_run = mt;
             l_run *= alpha;
           }
-          if (kt > x.lo[X]) {
+          if (kt > lo_x) {
             // O holds every PV up to tile kt-1 (the S-ready commit of this
             // tile covered them).
 #pragma unroll 1
@@ -578,7 +584,8 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx& c,
                                               const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                                              const CUtensorMap* tmV, uint32_t sQ0, uint32_t sK0,
+                                              const CUtensorMap* tmV, const CUtensorMap* tmKw,
+                                              const CUtensorMap* tmVw, uint32_t sQ0, uint32_t sK0,
                                               uint32_t sV0) {
   Ring kr, vr;
   uint32_t nq = 0;
@@ -597,8 +604,11 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
     if (!c.wait(B_KEMPTY0 + ks, kr.phase ^ 1)) return false;
     kr.next(kKStages);
     mbar_expect_tx(c.bar(B_KFULL0 + ks), kTileBytes);
-    tma_load_3d(sK0 + ks * kTileBytes, tmK, c.bar(B_KFULL0 + ks), 0, kt * 128, zk);
-    tma_load_3d(sK0 + ks * kTileBytes + kHalfBytes, tmK, c.bar(B_KFULL0 + ks), 64, kt * 128, zk);
+    const bool win = kt * 128 < p.q_off;
+    const CUtensorMap* mk = win ? tmKw : tmK;
+    const int row = win ? kt * 128 : kt * 128 - p.q_off;
+    tma_load_3d(sK0 + ks * kTileBytes, mk, c.bar(B_KFULL0 + ks), 0, row, zk);
+    tma_load_3d(sK0 + ks * kTileBytes + kHalfBytes, mk, c.bar(B_KFULL0 + ks), 64, row, zk);
     return true;
   };
   auto load_v = [&](int kt, int zk) -> bool {
@@ -606,8 +616,11 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
     if (!c.wait(B_VEMPTY0 + vs, vr.phase ^ 1)) return false;
     vr.next(kVStages);
     mbar_expect_tx(c.bar(B_VFULL0 + vs), kTileBytes);
-    tma_load_3d(sV0 + vs * kTileBytes, tmV, c.bar(B_VFULL0 + vs), 0, kt * 128, zk);
-    tma_load_3d(sV0 + vs * kTileBytes + kHalfBytes, tmV, c.bar(B_VFULL0 + vs), 64, kt * 128, zk);
+    const bool win = kt * 128 < p.q_off;
+    const CUtensorMap* mv = win ? tmVw : tmV;
+    const int row = win ? kt * 128 : kt * 128 - p.q_off;
+    tma_load_3d(sV0 + vs * kTileBytes, mv, c.bar(B_VFULL0 + vs), 0, row, zk);
+    tma_load_3d(sV0 + vs * kTileBytes + kHalfBytes, mv, c.bar(B_VFULL0 + vs), 64, row, zk);
     return true;
   };
   for (uint32_t i = 0;; ++i) {
@@ -659,6 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
+                          const __grid_constant__ CUtensorMap tmKw,
+                          const __grid_constant__ CUtensorMap tmVw,
                           const __grid_constant__ PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -687,6 +702,10 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if (p.q_off > 0) {
+      prefetch_tmap(&tmKw);
+      prefetch_tmap(&tmVw);
+    }
   }
   if (warp == 0) tmem_alloc(smem_addr((const void*)tmem_slot), kTmemCols);
   tc_fence_before();
@@ -697,7 +716,7 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp < 4) {
     if constexpr (kRegsControl < kRegsLaunch) regs_dec<kRegsControl>();
     if (warp == 0 && lane == 0)
-      producer_role(p, c, &tmQ, &tmK, &tmV, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
+      producer_role(p, c, &tmQ, &tmK, &tmV, &tmKw, &tmVw, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
     else if (warp == 2 && lane == 0)
       fetcher_role(p, c);
     else if (warp == 1 && lane == 0)
@@ -831,19 +850,29 @@ size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
 
 namespace {
 
-// Query rows 0 .. Nq-1 are key positions q_off .. q_off+Nq-1 of key rows
-// 0 .. Nk-1 (q_off a multiple of 128); t: per-sequence token counts of a
-// chunk (rows below q_off - t[b] masked), or nullptr for a prompt.
-moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, void* o, int32_t B,
-                                    int32_t Hq, int32_t Hkv, int32_t Nq, int32_t Nk, int32_t q_off,
-                                    const int64_t* t, const int32_t* spans, float scale, void* ws,
-                                    size_t ws_bytes, cudaStream_t s) {
+// Query rows 0 .. Nq-1 are key positions q_off .. q_off+Nq-1 (q_off a
+// multiple of 128).  Key rows q_off .. q_off+Nq-1 are k, v [B, Hkv, Nq, d];
+// rows 0 .. q_off-1 are kw, vw [B, Hkv, q_off, d].  t: per-sequence token
+// counts of a chunk (rows below q_off - t[b] masked), or nullptr for a prompt
+// (q_off = 0).
+moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, const void* kw,
+                                    const void* vw, void* o, int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq,
+                                    int32_t q_off, const int64_t* t, const int32_t* spans, float scale,
+                                    void* ws, size_t ws_bytes, cudaStream_t s) {
   if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, Nq, (int64_t)B * Hq) || !make_map(&mk, k, Nk, (int64_t)B * Hkv) ||
-      !make_map(&mv, v, Nk, (int64_t)B * Hkv))
+  const int32_t Nk = q_off + Nq;
+  CUtensorMap mq, mk, mv, mkw, mvw;
+  if (!make_map(&mq, q, Nq, (int64_t)B * Hq) || !make_map(&mk, k, Nq, (int64_t)B * Hkv) ||
+      !make_map(&mv, v, Nq, (int64_t)B * Hkv))
     return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
+  if (q_off > 0) {
+    if (!make_map(&mkw, kw, q_off, (int64_t)B * Hkv) || !make_map(&mvw, vw, q_off, (int64_t)B * Hkv))
+      return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
+  } else {
+    mkw = mk;                                      // never read: no key row lies below q_off
+    mvw = mv;
+  }
   // Header (error word, zeroed), the per-CTA list offsets and the units,
   // uploaded in one copy.  The pageable source is staged by the runtime
   // before cudaMemcpyAsync returns.
@@ -880,15 +909,15 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "prefill smem attribute");
-  prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, p);
+  prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mkw, mvw, p);
   return check_launch("prefill_bf16 launch");
 }
 
-// Chunk workspace: the prefill schedule region, then the gathered key and
-// value rows [B, Hkv, W + n, d] (W = prior keys any query can reach,
+// Chunk workspace: the prefill schedule region, then the gathered window
+// key and value rows [B, Hkv, W, d] (W = prior keys any query can reach,
 // rounded up to a tile).
 struct ChunkLayout {
-  int32_t W = 0, Nk = 0;
+  int32_t W = 0;
   size_t off_k = 0, off_v = 0, bytes = 0;
 };
 
@@ -897,8 +926,7 @@ ChunkLayout chunk_layout(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const in
   int32_t max_s = 1;
   for (int h = 0; h < Hq; ++h) max_s = std::max(max_s, spans[h]);
   L.W = (max_s - 1 + kTileN - 1) / kTileN * kTileN;
-  L.Nk = L.W + n;
-  const size_t rows = (size_t)B * Hkv * (size_t)L.Nk * kD * 2;
+  const size_t rows = (size_t)B * Hkv * (size_t)L.W * kD * 2;
   L.off_k = (prefill_workspace_bytes(B, Hq, n) + 255) / 256 * 256;
   L.off_v = L.off_k + (rows + 255) / 256 * 256;
   L.bytes = L.off_v + rows;
@@ -910,7 +938,8 @@ ChunkLayout chunk_layout(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const in
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
                                int32_t Hq, int32_t Hkv, int32_t N, const int32_t* spans, float scale,
                                void* ws, size_t ws_bytes, cudaStream_t s) {
-  return launch_prefill_bf16_rows(q, k, v, o, B, Hq, Hkv, N, N, 0, nullptr, spans, scale, ws, ws_bytes, s);
+  return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, B, Hq, Hkv, N, 0, nullptr, spans, scale, ws,
+                                  ws_bytes, s);
 }
 
 size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans) {
@@ -924,10 +953,13 @@ moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, c
   if (ws_bytes < L.bytes) return MOA_ERR_WORKSPACE;
   char* sk = static_cast<char*>(ws) + L.off_k;
   char* sv = static_cast<char*>(ws) + L.off_v;
-  moa_status st = launch_gather_window(c, k, v, n, L.W, sk, sv, s);
-  if (st != MOA_OK) return st;
+  moa_status st = MOA_OK;
+  if (L.W > 0) {
+    st = launch_gather_window(c, L.W, sk, sv, s);
+    if (st != MOA_OK) return st;
+  }
   const int64_t* t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
-  st = launch_prefill_bf16_rows(q, sk, sv, o, c->B, Hq, c->Hkv, n, L.Nk, L.W, t, spans, scale, ws, L.off_k, s);
+  st = launch_prefill_bf16_rows(q, k, v, sk, sv, o, c->B, Hq, c->Hkv, n, L.W, t, spans, scale, ws, L.off_k, s);
   if (st != MOA_OK) return st;
   return launch_append(c, k, v, n, s);
 }

@@ -210,11 +210,13 @@ moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t*
  *   spans: host int32[Hq], 1 <= spans[h] <= C_{h/(Hq/Hkv)}, else
  *   MOA_ERR_CAPACITY.
  *   workspace: moa_chunk_workspace_bytes(...) bytes, 256-byte aligned, no
- *   initialisation needed; it holds the work-unit schedule and the gathered
- *   key/value rows [B, Hkv, W + n, d], W = max_h S_h - 1 rounded up to 128.
- * Three launches on `stream`: the window gather, the tensor-core prefill
- * kernel (query rows offset by W into the gathered rows, rows of negative
- * positions masked), the append.  Errors as moa_prefill. */
+ *   initialisation needed; it holds the work-unit schedule and the window's
+ *   key/value rows gathered from the ring, [B, Hkv, W, d] with
+ *   W = max_h S_h - 1 rounded up to 128.
+ * Three launches on `stream` (two when every span is 1): the window gather,
+ * the tensor-core prefill kernel (key tiles below W from the gathered rows,
+ * the chunk's own straight from k, v; rows of negative positions masked),
+ * the append.  Errors as moa_prefill. */
 moa_status moa_chunk_workspace_bytes(const moa_kv_cache* cache, int32_t Hq, int32_t n,
                                      const int32_t* spans, size_t* bytes_out);
 moa_status moa_prefill_chunk(moa_kv_cache* cache, const void* q, const void* k, const void* v,
