@@ -28,7 +28,7 @@ namespace {
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kChunk = 512;          // window entries per split
-constexpr int kUnroll = 8;           // rows per batch: 2*kUnroll 16-byte loads in flight
+constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
 
 struct DecodeParams {
   char* data;                        // cache data region
