@@ -646,3 +646,85 @@ def test_prefill_chunk_errors():
         moa.moa_prefill_chunk(cache.handle, q, kv, kv, q.clone(), 4, 0, spans, 0.088, ptr, nb)
     assert e.value.status == moa.MOA_ERR_INVALID_ARG
     assert cache.positions() == [0]
+
+
+# ---------------------------------------------------------------------------
+# Largest head count the ABI takes (MOA_MAX_HEADS = 128) and a large batch
+# ---------------------------------------------------------------------------
+def test_bf16_prefill_at_the_head_limit():
+    """128 query heads on 8 KV heads (16 per group), ragged N, spans from 1 to
+    beyond N: every output row against the oracle."""
+    B, Hq, Hkv, N, d = 1, 128, 8, 300, 128
+    rng = np.random.default_rng(11)
+    spans = [int(s) for s in rng.integers(1, 400, Hq)]
+    spans[0], spans[1], spans[-1] = 1, 300, 399
+    q = inputs.randn(160, (B, Hq, N, d))
+    k = inputs.randn(161, (B, Hkv, N, d))
+    v = inputs.randn(162, (B, Hkv, N, d))
+    o = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, 1 / math.sqrt(d))
+    want = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, 1 / math.sqrt(d))
+    assert np.max(np.abs(inputs.as_f64(o) - want)) <= BF16_TOL
+
+
+def test_bf16_decode_at_the_head_limit():
+    """128 query heads on 16 KV heads (8 per group), three fused steps.  The
+    windows overlap enough (the sum of the spans is well above 2.2 times the
+    sum of the group capacities) for the group-shared decode kernel; half of
+    the groups hold near-equal windows, the other half spans from 1 to 700."""
+    B, Hq, Hkv, d, prefix = 2, 128, 16, 128, 700
+    rng = np.random.default_rng(12)
+    spans = [int(s) for s in rng.integers(1, 701, Hq)]
+    for h in range(0, 64):            # first half of the groups: near-equal windows (group kernel)
+        spans[h] = 600 + (h % 8) * 12
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    k0 = inputs.randn(170, (B, Hkv, prefix, d))
+    v0 = inputs.randn(171, (B, Hkv, prefix, d))
+    cache.append(k0.to(DEV), v0.to(DEV))
+    ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    for step in range(3):
+        qt = inputs.randn(180 + step, (B, Hq, d))
+        kt = inputs.randn(185 + step, (B, Hkv, 1, d))
+        vt = inputs.randn(190 + step, (B, Hkv, 1, d))
+        ot = _nan_like((B, Hq, d), torch.bfloat16)
+        moa.moa_decode_append(cache.handle, qt.to(DEV), kt.to(DEV), vt.to(DEV), ot, Hq, spans, scale, ws.ptr,
+                              ws.nbytes)
+        torch.cuda.synchronize()
+        ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+        ref = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+        assert np.max(np.abs(inputs.as_f64(ot) - ref)) <= BF16_TOL, step
+    assert cache.positions() == ring.t
+
+
+def test_bf16_decode_large_batch_sampled():
+    """1024 sequences at different positions (set through moa_kv_set_positions
+    over caches filled in one append): per-sequence counters and positions,
+    sampled sequences against the oracle."""
+    B, Hq, Hkv, d, prefix = 1024, 4, 2, 128, 96
+    spans = [1, 37, 96, 64]
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    k0 = inputs.randn_cuda(200, (B, Hkv, prefix, d))
+    v0 = inputs.randn_cuda(201, (B, Hkv, prefix, d))
+    cache.append(k0, v0)
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    q = inputs.randn_cuda(202, (B, Hq, d))
+    kn = inputs.randn_cuda(203, (B, Hkv, 1, d))
+    vn = inputs.randn_cuda(204, (B, Hkv, 1, d))
+    o = _nan_like((B, Hq, d), torch.bfloat16)
+    moa.moa_decode_append(cache.handle, q, kn, vn, o, Hq, spans, scale, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    assert cache.positions() == [prefix + 1] * B
+    assert torch.isfinite(o.float()).all()
+    kf, vf, qf = inputs.as_f64(k0), inputs.as_f64(v0), inputs.as_f64(q)
+    knf, vnf = inputs.as_f64(kn), inputs.as_f64(vn)
+    got = inputs.as_f64(o)
+    for b in [0, 1, 511, 777, B - 1]:
+        hist_k = np.concatenate([kf[b], knf[b]], axis=1)
+        hist_v = np.concatenate([vf[b], vnf[b]], axis=1)
+        want = oatt.chunk(qf[b:b + 1, :, None, :], [hist_k], [hist_v], [prefix], spans, scale)[0, :, 0]
+        assert np.max(np.abs(got[b] - want)) <= BF16_TOL, b
