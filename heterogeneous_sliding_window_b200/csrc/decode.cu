@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace moa {
 namespace {
@@ -338,8 +339,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
   const T* vn = fused ? reinterpret_cast<const T*>(p.v_new) + ((size_t)b * Hkv + g) * D : nullptr;
 
   // head j of the group sees window entries e >= e0[j] (e counts from the
-  // oldest entry of the group's window)
-  float qf[G][VE];
+  // oldest entry of the group's window).  q is held as f32 pairs.
+  using sm100::f2_pack;
+  using sm100::f2_unpack;
+  using sm100::f2_fma;
+  using sm100::f2_add;
+  uint64_t q2[G][VE / 2];
   int e0[G];
 #pragma unroll
   for (int j = 0; j < G; ++j) {
@@ -348,19 +353,34 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
     e0[j] = W - Sh;
     const int4 raw = __ldg(reinterpret_cast<const int4*>(
         reinterpret_cast<const T*>(p.q) + ((size_t)b * p.Hq + h) * D + li * VE));
-    Vec16<T>::cvt(raw, qf[j]);
+    float qf[VE];
+    Vec16<T>::cvt(raw, qf);
 #pragma unroll
-    for (int e = 0; e < VE; ++e) qf[j][e] *= p.scale_log2;
+    for (int e = 0; e < VE / 2; ++e) q2[j][e] = f2_pack(qf[2 * e] * p.scale_log2, qf[2 * e + 1] * p.scale_log2);
   }
+  // After the transposing reduction below, lane li of a row group holds the
+  // full score of head hj = li >> kShift (LPR / G lanes per head).
+  constexpr int kLogG = G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
+  static_assert((1 << kLogG) == G && G <= LPR, "group size");
+  constexpr int kLogL = LPR == 32 ? 5 : LPR == 16 ? 4 : LPR == 8 ? 3 : LPR == 4 ? 2 : LPR == 2 ? 1 : 0;
+  static_assert((1 << kLogL) == LPR, "lanes per row");
+  constexpr int kShift = kLogL - kLogG;
+  const int hj = li >> kShift;
+  const int e0_own = [&] {
+    int v = 0;
+#pragma unroll
+    for (int j = 0; j < G; ++j) if (j == hj) v = e0[j];
+    return v;
+  }();
+  const int lane0 = sub * LPR;                          // first lane of this row group
 
-  float m[G], l[G], acc[G][VE];
+  // running max and sum of head hj (this lane's), accumulators of every head
+  float m_own = -INFINITY, l_own = 0.f;
+  uint64_t acc2[G][VE / 2];
 #pragma unroll
-  for (int j = 0; j < G; ++j) {
-    m[j] = -INFINITY;
-    l[j] = 0.f;
+  for (int j = 0; j < G; ++j)
 #pragma unroll
-    for (int e = 0; e < VE; ++e) acc[j][e] = 0.f;
-  }
+    for (int e = 0; e < VE / 2; ++e) acc2[j][e] = 0;
 
   // The trip count is uniform across the CTA (every lane takes part in the
   // shuffles below); rows past the chunk are masked instead.
@@ -386,46 +406,81 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
         vr[u] = make_int4(0, 0, 0, 0);
       }
     }
-    float sv[G][U];
+    // scores: G partial dot products per lane, then a reduction over the row
+    // group's lanes that halves the number of values at each of the first
+    // kLogG levels, so each lane ends with one head's full sum
+    float s_own[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float kf[VE];
       Vec16<T>::cvt(kr[u], kf);
-      const int row = base + u * NG + grp;
+      float d[G];
 #pragma unroll
       for (int j = 0; j < G; ++j) {
-        float dot = 0.f;
+        uint64_t a2 = 0;
 #pragma unroll
-        for (int e = 0; e < VE; ++e) dot = fmaf(qf[j][e], kf[e], dot);
-#pragma unroll
-        for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        sv[j][u] = (row < nrows && w0 + row >= e0[j]) ? dot : -INFINITY;
+        for (int e = 0; e < VE / 2; ++e) a2 = f2_fma(q2[j][e], f2_pack(kf[2 * e], kf[2 * e + 1]), a2);
+        float x0, x1;
+        f2_unpack(a2, x0, x1);
+        d[j] = x0 + x1;
       }
+      int n = G;
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) {
+        if (n > 1) {
+          const bool up = (li & off) != 0;
+#pragma unroll
+          for (int k = 0; k < n / 2; ++k) {
+            const float send = up ? d[k] : d[k + n / 2];
+            const float keep = up ? d[k + n / 2] : d[k];
+            d[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+          }
+          n >>= 1;
+        } else {
+          d[0] += __shfl_xor_sync(0xffffffffu, d[0], off);
+        }
+      }
+      const int row = base + u * NG + grp;
+      s_own[u] = (row < nrows && w0 + row >= e0_own) ? d[0] : -INFINITY;
     }
+    // online softmax of head hj over the batch
+    float bmax = m_own;
+#pragma unroll
+    for (int u = 0; u < U; ++u) bmax = fmaxf(bmax, s_own[u]);
+    // 0 when the max moves up from -inf, 1 when unchanged (also while still -inf)
+    const float corr_own = bmax == m_own ? 1.f : exp2f(m_own - bmax);
+    m_own = bmax;
+    // a head that has seen no row yet keeps m = -inf: p = 0, not NaN
+    const float mref = m_own == -INFINITY ? 0.f : m_own;
+    float p_own[U];
+    l_own *= corr_own;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      p_own[u] = exp2f(s_own[u] - mref);
+      l_own += p_own[u];
+    }
+    // every lane updates the accumulators of every head: correction factors
+    // and weights come from the lanes that own each head
 #pragma unroll
     for (int j = 0; j < G; ++j) {
-      float bmax = m[j];
+      const float cj = __shfl_sync(0xffffffffu, corr_own, lane0 + (j << kShift));
+      const uint64_t c2 = f2_pack(cj, cj);
 #pragma unroll
-      for (int u = 0; u < U; ++u) bmax = fmaxf(bmax, sv[j][u]);
-      if (bmax > m[j]) {                               // uniform across the group's lanes
-        const float corr = exp2f(m[j] - bmax);         // 0 when m = -inf
-        l[j] *= corr;
-#pragma unroll
-        for (int e = 0; e < VE; ++e) acc[j][e] *= corr;
-        m[j] = bmax;
-      }
+      for (int e = 0; e < VE / 2; ++e) acc2[j][e] = f2_fma(acc2[j][e], c2, 0);
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float vf[VE];
       Vec16<T>::cvt(vr[u], vf);
+      uint64_t v2[VE / 2];
+#pragma unroll
+      for (int e = 0; e < VE / 2; ++e) v2[e] = f2_pack(vf[2 * e], vf[2 * e + 1]);
 #pragma unroll
       for (int j = 0; j < G; ++j) {
-        // a head that has seen no row yet keeps m = -inf: p = 0, not NaN
-        const float pu = exp2f(sv[j][u] - (m[j] == -INFINITY ? 0.f : m[j]));
-        l[j] += pu;
+        const float pj = __shfl_sync(0xffffffffu, p_own[u], lane0 + (j << kShift));
+        const uint64_t p2 = f2_pack(pj, pj);
 #pragma unroll
-        for (int e = 0; e < VE; ++e) acc[j][e] = fmaf(pu, vf[e], acc[j][e]);
+        for (int e = 0; e < VE / 2; ++e) acc2[j][e] = f2_fma(p2, v2[e], acc2[j][e]);
       }
     }
   }
@@ -434,10 +489,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
 #pragma unroll
   for (int j = 0; j < G; ++j) {
 #pragma unroll
-    for (int e = 0; e < VE; ++e) g_acc[grp][li * VE + e] = acc[j][e];
-    if (li == 0) {
-      g_m[grp] = m[j];
-      g_l[grp] = l[j];
+    for (int e = 0; e < VE / 2; ++e) f2_unpack(acc2[j][e], g_acc[grp][li * VE + 2 * e], g_acc[grp][li * VE + 2 * e + 1]);
+    if (li == (j << kShift)) {
+      g_m[grp] = m_own;
+      g_l[grp] = l_own;
     }
     __syncthreads();
     float M = -INFINITY;
