@@ -30,6 +30,14 @@ constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kChunk = 512;          // window entries per split
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
+#ifndef MOA_GROUP_MMA
+#define MOA_GROUP_MMA 1
+#endif
+constexpr bool kGroupMma = MOA_GROUP_MMA != 0;   // tensor-core group kernel for bf16, d = 128
+#ifndef MOA_GROUP_MMA2
+#define MOA_GROUP_MMA2 1
+#endif
+constexpr bool kGroupMma2 = MOA_GROUP_MMA2 != 0; // ... also for two query heads per KV head
 
 struct DecodeParams {
   char* data;                        // cache data region
@@ -557,6 +565,329 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Grouped-query decode on the tensor cores (bf16, d = 128).
+//
+// Same work item, window geometry and partial layout as decode_group_kernel:
+// one CTA per (b, KV group g, split of kChunk group-window entries).  Warp w
+// takes entries [128w, 128w + 128) of the split in tiles of 16 cached rows:
+//   * cp.async copies the tile's K and V rows (16 x 256 bytes each) into a
+//     two-stage per-warp buffer, 16-byte chunks XOR-swizzled by row so that
+//     ldmatrix reads them without bank conflicts;
+//   * S^T[16 rows x 8 heads] = K_tile . Q_g^T with mma.m16n8k16 (A = K from
+//     ldmatrix, B = the group's q held in registers; heads past G are zero);
+//   * per head an online softmax over the rows (each lane holds heads
+//     2(lane%4), 2(lane%4)+1 for rows lane/4 and lane/4 + 8);
+//   * P goes through a 256-byte per-warp scratch into the B-operand layout,
+//     and O^T[128 dims x 8 heads] += V_tile^T . P^T (A = V from ldmatrix.trans).
+// The four warps then merge by log-sum-exp in shared memory and the split's
+// partial (m, l, o) per head is written or, with one split, o itself.
+constexpr int kMmaRows = 16;                      // cached rows per tile
+constexpr int kMmaTileBytes = kMmaRows * 128 * 2; // one 16 x 128 bf16 tile
+constexpr int kMmaWarpRows = kChunk / kDecWarps;  // entries per warp and split
+constexpr size_t kMmaSmem = (size_t)kDecWarps * (2 * 2 * kMmaTileBytes + 256);   // tiles + P scratch
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// d[0..3] += A[16x16] . B[16x8], bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// byte offset of 16-byte chunk c of row r in a swizzled 16 x 256-byte tile
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4)); }
+
+template <int G>
+__global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int D = 128;
+  static_assert(G == 2 || G == 4 || G == 8, "group size");
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ int last_flag;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int g4 = lane >> 2, c4 = lane & 3;
+
+  const int item = blockIdx.x;
+  const int b = item / p.items_per_b;
+  const int r = item - b * p.items_per_b;
+  const int Hkv = p.Hq / G;
+  int lo = 0, hi = Hkv - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.split_pre[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  const int g = lo;
+  const int s = r - p.split_pre[g];
+  const int nsplit = p.split_pre[g + 1] - p.split_pre[g];
+  const int C = p.cap[g];
+  const bool fused = p.k_new != nullptr;
+  const int64_t t0 = p.t[b];
+  if (fused) step_counted(p, b, t0);
+  const int64_t tb = fused ? t0 + 1 : t0;
+  const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);
+  const int w0 = s * kChunk;
+  const int nrows = max(0, min(kChunk, W - w0));
+  const int64_t pos0 = tb - W + w0;
+  const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
+  const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
+  const __nv_bfloat16* Vb = Kb + (size_t)C * D;
+  const int e_new = fused ? W - 1 : -1;
+  const __nv_bfloat16* kn = fused ? reinterpret_cast<const __nv_bfloat16*>(p.k_new) + ((size_t)b * Hkv + g) * D : nullptr;
+  const __nv_bfloat16* vn = fused ? reinterpret_cast<const __nv_bfloat16*>(p.v_new) + ((size_t)b * Hkv + g) * D : nullptr;
+
+  // B operand of S^T: q of head n = lane/4 (zero past G), dims 16kk + 2(lane%4) + {0,1} and + {8,9}
+  uint32_t qb[8][2];
+  {
+    const bool hv = g4 < G;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+        reinterpret_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * G + (hv ? g4 : 0)) * D);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qb[kk][0] = hv ? __ldg(qrow + 8 * kk + c4) : 0u;
+      qb[kk][1] = hv ? __ldg(qrow + 8 * kk + c4 + 4) : 0u;
+    }
+  }
+  // heads this lane owns in the accumulator layouts, and where their windows start
+  const int h0 = 2 * c4, h1 = 2 * c4 + 1;
+  int e0a = 1 << 30, e0b = 1 << 30;              // past every entry: heads beyond G see no row
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const int Sh = (int)(tb < (int64_t)p.span[g * G + j] ? tb : (int64_t)p.span[g * G + j]);
+    if (j == h0) e0a = W - Sh;
+    if (j == h1) e0b = W - Sh;
+  }
+
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsm) + (uint32_t)warp * (2 * 2 * kMmaTileBytes + 256);
+  const uint32_t sP = sbase + 2 * 2 * kMmaTileBytes;             // [8 heads][16 rows] bf16
+  uint16_t* sPg = reinterpret_cast<uint16_t*>(dsm + (size_t)warp * (2 * 2 * kMmaTileBytes + 256) + 2 * 2 * kMmaTileBytes);
+  const int wrow0 = warp * kMmaWarpRows;                          // first split entry of this warp
+  const int wrows = max(0, min(kMmaWarpRows, nrows - wrow0));
+  const int ntiles = (wrows + kMmaRows - 1) / kMmaRows;
+
+  // issue the copies of tile ti into stage st (rows past the split are zero-filled)
+  auto load_tile = [&](int ti, int st) {
+    const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = lane + 32 * q;
+      const int rr = i >> 4, cc = i & 15;
+      const int row = wrow0 + ti * kMmaRows + rr;                // split entry
+      const __nv_bfloat16* srcK = Kb;
+      const __nv_bfloat16* srcV = Vb;
+      uint32_t bytes = 0;
+      if (row < nrows) {
+        bytes = 16;
+        if (w0 + row == e_new) {
+          srcK = kn + cc * 8;
+          srcV = vn + cc * 8;
+          int slot = slot0 + row;
+          if (slot >= C) slot -= C;
+          // this CTA is the group's only reader of the newest entry: write it to its slot
+          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Kb) + (size_t)slot * D + cc * 8) =
+              __ldg(reinterpret_cast<const int4*>(srcK));
+          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Vb) + (size_t)slot * D + cc * 8) =
+              __ldg(reinterpret_cast<const int4*>(srcV));
+        } else {
+          int slot = slot0 + row;
+          if (slot >= C) slot -= C;
+          srcK = Kb + (size_t)slot * D + cc * 8;
+          srcV = Vb + (size_t)slot * D + cc * 8;
+        }
+      }
+      cp_async16(dK + swz(rr, cc), srcK, bytes);
+      cp_async16(dV + swz(rr, cc), srcV, bytes);
+    }
+  };
+
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h1
+  float oacc[8][4];
+#pragma unroll
+  for (int mb = 0; mb < 8; ++mb)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[mb][e] = 0.f;
+
+  if (ntiles > 0) load_tile(0, 0);
+  cp_async_commit();
+  for (int ti = 0; ti < ntiles; ++ti) {
+    if (ti + 1 < ntiles) load_tile(ti + 1, (ti + 1) & 1);
+    cp_async_commit();
+    cp_async_wait1();
+    __syncwarp();
+    const uint32_t tK = sbase + (uint32_t)(ti & 1) * 2 * kMmaTileBytes, tV = tK + kMmaTileBytes;
+    // S^T = K . Q^T
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int ar = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(tK + swz(ar, 2 * kk + (lane >> 4)), a);
+        mma16816(sacc, a, qb[kk][0], qb[kk][1]);
+      }
+    }
+    // mask and scale: rows g4 and g4 + 8 of the tile, heads h0 and h1
+    const int ra = wrow0 + ti * kMmaRows + g4, rb = ra + 8;
+    const float sc = p.scale_log2;
+    const float s0 = (ra < nrows && w0 + ra >= e0a) ? sacc[0] * sc : -INFINITY;
+    const float s1 = (ra < nrows && w0 + ra >= e0b) ? sacc[1] * sc : -INFINITY;
+    const float s2 = (rb < nrows && w0 + rb >= e0a) ? sacc[2] * sc : -INFINITY;
+    const float s3 = (rb < nrows && w0 + rb >= e0b) ? sacc[3] * sc : -INFINITY;
+    float t0m = fmaxf(s0, s2), t1m = fmaxf(s1, s3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      t0m = fmaxf(t0m, __shfl_xor_sync(0xffffffffu, t0m, off));
+      t1m = fmaxf(t1m, __shfl_xor_sync(0xffffffffu, t1m, off));
+    }
+    const float n0 = fmaxf(m0, t0m), n1 = fmaxf(m1, t1m);
+    const float cr0 = n0 == m0 ? 1.f : exp2f(m0 - n0);        // 0 when m was -inf
+    const float cr1 = n1 == m1 ? 1.f : exp2f(m1 - n1);
+    m0 = n0;
+    m1 = n1;
+    const float r0 = m0 == -INFINITY ? 0.f : m0, r1 = m1 == -INFINITY ? 0.f : m1;
+    const float p0 = exp2f(s0 - r0), p1 = exp2f(s1 - r1), p2 = exp2f(s2 - r0), p3 = exp2f(s3 - r1);
+    l0 = l0 * cr0 + p0 + p2;
+    l1 = l1 * cr1 + p1 + p3;
+#pragma unroll
+    for (int mb = 0; mb < 8; ++mb) {
+      oacc[mb][0] *= cr0;
+      oacc[mb][1] *= cr1;
+      oacc[mb][2] *= cr0;
+      oacc[mb][3] *= cr1;
+    }
+    // P^T into the B-operand layout through the scratch [head][row]
+    sPg[h0 * 16 + g4] = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
+    sPg[h1 * 16 + g4] = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
+    sPg[h0 * 16 + g4 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(p2));
+    sPg[h1 * 16 + g4 + 8] = __bfloat16_as_ushort(__float2bfloat16_rn(p3));
+    __syncwarp();
+    uint32_t pb0, pb1;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb0) : "r"(sP + (uint32_t)(g4 * 32 + c4 * 4)));
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(pb1) : "r"(sP + (uint32_t)(g4 * 32 + c4 * 4 + 16)));
+    // O^T += V^T . P^T
+    {
+      const int vr = (lane & 7) + ((lane >> 4) & 1) * 8;
+#pragma unroll
+      for (int mb = 0; mb < 8; ++mb) {
+        uint32_t a[4];
+        ldsm_x4_t(tV + swz(vr, 2 * mb + ((lane >> 3) & 1)), a);
+        mma16816(oacc[mb], a, pb0, pb1);
+      }
+    }
+    __syncwarp();                                       // stage and scratch are rewritten next
+  }
+  cp_async_wait0();
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+
+  // merge the four warps: per warp m, l [8 heads] and o [8 heads][128] in fp32
+  __syncthreads();
+  float* mw = reinterpret_cast<float*>(dsm);                  // [4][8]
+  float* lw = mw + kDecWarps * 8;                             // [4][8]
+  float* ow = lw + kDecWarps * 8;                             // [4][8][128]
+  if (g4 == 0) {
+    mw[warp * 8 + h0] = m0;
+    mw[warp * 8 + h1] = m1;
+    lw[warp * 8 + h0] = l0;
+    lw[warp * 8 + h1] = l1;
+  }
+#pragma unroll
+  for (int mb = 0; mb < 8; ++mb) {
+    float* o = ow + warp * 8 * D;
+    o[h0 * D + 16 * mb + g4] = oacc[mb][0];
+    o[h1 * D + 16 * mb + g4] = oacc[mb][1];
+    o[h0 * D + 16 * mb + g4 + 8] = oacc[mb][2];
+    o[h1 * D + 16 * mb + g4 + 8] = oacc[mb][3];
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int j = 0; j < G; ++j) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, mw[w * 8 + j]);
+    float L = 0.f, od = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kDecWarps; ++w) {
+        const float wt = exp2f(mw[w * 8 + j] - M);
+        L = fmaf(wt, lw[w * 8 + j], L);
+        od = fmaf(wt, ow[(w * 8 + j) * D + tid], od);
+      }
+    }
+    const int h = g * G + j;
+    if (nsplit == 1) {
+      reinterpret_cast<__nv_bfloat16*>(p.o)[((size_t)b * p.Hq + h) * D + tid] = __float2bfloat16_rn(L > 0.f ? od / L : 0.f);
+    } else {
+      const size_t idx = (size_t)b * p.hslot_pre[p.Hq] + p.hslot_pre[h] + s;
+      p.part_o[idx * D + tid] = od;
+      if (tid == 0) {
+        p.part_ml[2 * idx] = M;
+        p.part_ml[2 * idx + 1] = L;
+      }
+    }
+  }
+  if (nsplit == 1) {
+    if (tid == 0 && W == 0) atomicOr(p.err, kErrEmpty);
+    return;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned prev = atomicAdd(&p.ctr[(size_t)b * p.Hq + g], 1u);
+    last_flag = (prev == (unsigned)(nsplit - 1));
+  }
+  __syncthreads();
+  if (!last_flag) return;
+  __threadfence();
+#pragma unroll 1
+  for (int j = 0; j < G; ++j) {
+    const int h = g * G + j;
+    const size_t first = (size_t)b * p.hslot_pre[p.Hq] + p.hslot_pre[h];
+    float MM = -INFINITY;
+    for (int ss = 0; ss < nsplit; ++ss) MM = fmaxf(MM, __ldcg(&p.part_ml[2 * (first + ss)]));
+    float LL = 0.f, A = 0.f;
+    if (MM != -INFINITY) {
+      for (int ss = 0; ss < nsplit; ++ss) {
+        const float ms = __ldcg(&p.part_ml[2 * (first + ss)]);
+        const float wt = exp2f(ms - MM);
+        LL = fmaf(wt, __ldcg(&p.part_ml[2 * (first + ss) + 1]), LL);
+        A = fmaf(wt, __ldcg(&p.part_o[(first + ss) * D + tid]), A);
+      }
+    }
+    reinterpret_cast<__nv_bfloat16*>(p.o)[((size_t)b * p.Hq + h) * D + tid] = __float2bfloat16_rn(LL > 0.f ? A / LL : 0.f);
+  }
+  if (tid == 0) {
+    p.ctr[(size_t)b * p.Hq + g] = 0u;
+    if (W == 0) atomicOr(p.err, kErrEmpty);
+  }
+}
+
+template <int G>
+cudaError_t launch_group_mma(const DecodeParams& p, unsigned grid, cudaStream_t s) {
+  static cudaError_t attr = cudaFuncSetAttribute(decode_group_mma_kernel<G>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMmaSmem);
+  if (attr != cudaSuccess) return attr;
+  decode_group_mma_kernel<G><<<grid, kDecThreads, kMmaSmem, s>>>(p);
+  return cudaGetLastError();
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_group(const DecodeParams& p, unsigned grid, cudaStream_t s) {
   decode_group_kernel<T, D, G><<<grid, kDecThreads, 0, s>>>(p);
@@ -639,17 +970,21 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
     p.cap[g] = c->cap[g];
     p.goff[g] = c->goff[g];
   }
-  // The group kernel reads each cached row once for all G heads but does G
-  // dot products and softmax updates per row; the per-head kernel reads
-  // overlapping windows once per head and L2 serves most of the repeats.  On
-  // a Llama3-8B-shaped layer (B=32, 32 query / 8 KV heads, context 8192) the
-  // group kernel was 5 % faster when the heads' windows summed to 2.24x the
-  // group windows and 8 % slower at 2.0x, so it is taken above 2.2x.
+  // The group kernels read each cached row once for all G heads; the
+  // per-head kernel reads overlapping windows once per head and L2 serves
+  // most of the repeats.  bf16 with d = 128 and G = 2, 4 or 8 always takes
+  // the tensor-core group kernel: on Llama3-8B-shaped layers (B=32, context
+  // 8192) it beat the per-head kernel at every overlap tried, down to heads'
+  // windows summing to 1.8x the group windows.  The SIMT group kernel (other
+  // types and sizes) does G dot products per row on the CUDA cores: it was
+  // 5 % faster than the per-head kernel at 2.24x and 8 % slower at 2.0x, so
+  // it is taken above 2.2x.
   const int G = Hq / c->Hkv;
   int64_t head_rows = 0, group_rows = 0;
   for (int h = 0; h < Hq; ++h) head_rows += spans[h];
   for (int g = 0; g < c->Hkv; ++g) group_rows += c->cap[g];
-  if ((G == 4 || G == 8) && head_rows * 10 > group_rows * 22) {
+  const bool mma_group = kGroupMma && c->dtype == MOA_BF16 && c->d == 128 && (G == 4 || G == 8 || (kGroupMma2 && G == 2));
+  if (mma_group || ((G == 4 || G == 8) && head_rows * 10 > group_rows * 22)) {
     // group kernel: splits per KV group over its capacity, G partial slots each
     int items = 0;
     p.split_pre[0] = 0;
@@ -664,7 +999,10 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
     const long long grid = (long long)c->B * items;
     if (grid > 0x7fffffffLL) return MOA_ERR_UNSUPPORTED;
     cudaError_t e;
-    if (c->dtype == MOA_BF16)
+    if (mma_group)
+      e = G == 2 ? launch_group_mma<2>(p, (unsigned)grid, s)
+                 : G == 4 ? launch_group_mma<4>(p, (unsigned)grid, s) : launch_group_mma<8>(p, (unsigned)grid, s);
+    else if (c->dtype == MOA_BF16)
       e = c->d == 128 ? launch_group_g<__nv_bfloat16, 128>(p, G, (unsigned)grid, s)
                       : launch_group_g<__nv_bfloat16, 64>(p, G, (unsigned)grid, s);
     else
