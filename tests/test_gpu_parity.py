@@ -322,6 +322,11 @@ FUSED_CASES = [
                                    2, 1000, 1024, 513, 257, 5, 1200, 40], 2),  # 8 heads per group
     (1, 4, 1, "bf16", 128, 2000, [1000, 513, 2000, 1], 2),                 # ring wraps
     (2, 4, 2, "f32", 64, 0, [1, 5, 32, 17], 40),                           # from an empty cache
+    # the SIMT group kernel (fp32 or d = 64 with 4 or 8 heads per KV head and
+    # windows overlapping more than 2.2x); bf16 d = 128 groups take the tensor-core kernel
+    (2, 8, 2, "f32", 64, 50, [40, 38, 40, 36, 64, 60, 64, 63], 3),
+    (2, 8, 2, "bf16", 64, 700, [600, 580, 512, 599, 64, 60, 64, 63], 3),
+    (1, 16, 2, "f32", 64, 30, [30, 29, 28, 27, 26, 25, 24, 23, 20, 20, 20, 20, 20, 20, 20, 19], 3),
 ]
 
 
