@@ -551,10 +551,11 @@ def gqa_decode_layer(stream, reps=20):
     ms = e0.elapsed_time(e1) / reps
     group_bytes = B * sum(2 * cp * D * 2 for cp in caps) + 2 * B * Hq * D * 2
     head_bytes = B * sum(2 * S * D * 2 for S in sp) + 2 * B * Hq * D * 2
-    group_path = sum(sp) * 10 > sum(caps) * 22
     c.close()
+    # bf16, d = 128 and 4 query heads per KV head: the tensor-core group kernel
     return {"workload": "llama3-8b-shaped decode layer: B=%d Hq=%d Hkv=%d d=%d ctx %d density 0.50" % (B, Hq, Hkv, D, N),
-            "kernel": "decode_group_kernel<bf16,128,4>" if group_path else "decode_kernel<bf16,128>",
+            "kernel": "decode_group_mma_kernel<%d> (bf16, d=128)" % G,
+            "frac_of_copy": round(group_bytes / (ms * 1e-3) / 1e9 / _peaks()[0], 4),
             "ms": round(ms, 4), "group_window_bytes": group_bytes, "per_head_window_bytes": head_bytes,
             "gbs_of_group_bytes": round(group_bytes / (ms * 1e-3) / 1e9, 1),
             "tokens_per_s_one_layer": round(B / (ms * 1e-3), 1)}
@@ -615,6 +616,8 @@ def run_profile_case(case, launches=3):
     decode : one decode layer of the 7B workload (B=32, 32 heads, context 4096; 1 GiB cache).
     chunk  : the bench's chunked prefill (4096-token chunk after 4096 cached tokens, 32 heads),
              `launches` calls of moa_prefill_chunk (gather, prefill kernel, append each).
+    gqa    : the bench's `gqa_decode` layer (Llama3-8B-shaped, B=32, 32/8 heads, context 8192,
+             50 %; 0.96 GB of group windows), `launches` decode calls.
     """
     import torch
     from heterogeneous_sliding_window_b200 import inputs, moa
@@ -631,6 +634,22 @@ def run_profile_case(case, launches=3):
             moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", sp, 1.0 / math.sqrt(P_D), ws.ptr,
                             ws.nbytes)
         moa.moa_workspace_check(ws.ptr)
+    elif case == "gqa":
+        B, Hq, Hkv, N, D = 32, 32, 8, 8192, 128
+        a, b = inputs.tables_7b(1001, Hq, N, BLOCK, 0.5, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, N, BLOCK)
+        G = Hq // Hkv
+        caps = [max(sp[g * G:(g + 1) * G]) for g in range(Hkv)]
+        c = moa.KVCache(B, Hkv, D, "bf16", caps)
+        data = c.data_bytes().view(torch.bfloat16)
+        data.copy_(inputs.randn_cuda(2000, (data.numel(),)))
+        c.set_positions([N] * B)
+        ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, D, sp)
+        q = inputs.randn_cuda(2001, (B, Hq, D))
+        o = torch.empty_like(q)
+        for _ in range(launches):
+            moa.moa_decode(c.handle, q, o, Hq, sp, 1.0 / math.sqrt(D), ws.ptr, ws.nbytes)
+        c.positions()
     elif case == "chunk":
         H, d, t, n = 32, 128, 4096, 4096
         a, b = inputs.tables_7b(P_SEED + 1, H, t + n, BLOCK, P_DENSITY, moa.moa_rules_eval)
@@ -669,7 +688,7 @@ def run_profile_case(case, launches=3):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-case", choices=["prefill", "decode", "chunk"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "chunk", "gqa"], default=None,
                     help="run one small single-kernel case (for ncu) and exit")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
