@@ -180,6 +180,14 @@ extern "C" moa_status moa_stream_read(const void* buf, size_t bytes, void* out, 
   return launch_stream_read(buf, bytes, out, (cudaStream_t)stream);
 }
 
+extern "C" moa_status moa_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* ws,
+                                             size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !o) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255u) != 0 || ws_bytes < prefill_workspace_bytes(1, 1, 128)) return MOA_ERR_WORKSPACE;
+  return launch_prefill_stall_test(q, k, v, o, ws, ws_bytes, (cudaStream_t)stream);
+}
+
 extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
                                            int32_t n_ctas, int32_t* rows_out, int64_t cap,
                                            int64_t* n_rows_out) {

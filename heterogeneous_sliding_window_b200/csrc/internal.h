@@ -87,6 +87,11 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
                                const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                cudaStream_t s);
 
+// Self-test of the prefill kernel's bounded waits (prefill_sm100.cu): one CTA
+// on a 1 x 1 x 128 x 128 problem whose unit records are never published.
+moa_status launch_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* ws,
+                                     size_t ws_bytes, cudaStream_t s);
+
 // Chunked prefill (prefill_sm100.cu): the n new tokens of every sequence
 // attend to the cache's window plus themselves, then are appended.
 size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans);

@@ -128,6 +128,7 @@ struct PrefillParams {
   int32_t N, Nq, q_off;
   const int64_t* t;
   int32_t Hq, Hkv, G;
+  int32_t stall;                 // self-test of the bounded waits: the fetcher publishes nothing
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
 };
@@ -650,6 +651,7 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
 // consumer, then a record with x < 0; no role waits on a global load.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void fetcher_role(const PrefillParams& p, const Ctx& c) {
+  if (p.stall) return;           // every other role's first wait runs out
   const int first = p.cta_off[blockIdx.x], last = p.cta_off[blockIdx.x + 1];
   for (uint32_t i = 0;; ++i) {
     const uint32_t slot = i % kUnitSlots;
@@ -858,7 +860,7 @@ namespace {
 moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, const void* kw,
                                     const void* vw, void* o, int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq,
                                     int32_t q_off, const int64_t* t, const int32_t* spans, float scale,
-                                    void* ws, size_t ws_bytes, cudaStream_t s) {
+                                    void* ws, size_t ws_bytes, cudaStream_t s, bool stall = false) {
   if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
   const int32_t Nk = q_off + Nq;
@@ -896,6 +898,7 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.Nq = Nq;
   p.q_off = q_off;
   p.t = t;
+  p.stall = stall ? 1 : 0;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -940,6 +943,13 @@ moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void
                                void* ws, size_t ws_bytes, cudaStream_t s) {
   return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, B, Hq, Hkv, N, 0, nullptr, spans, scale, ws,
                                   ws_bytes, s);
+}
+
+moa_status launch_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* ws,
+                                     size_t ws_bytes, cudaStream_t s) {
+  const int32_t span = 128;
+  return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, 1, 1, 1, 128, 0, nullptr, &span, 0.088f, ws,
+                                  ws_bytes, s, true);
 }
 
 size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans) {

@@ -25,7 +25,7 @@ EXPORTS = (
     "moa_kv_free", "moa_kv_append", "moa_kv_positions", "moa_kv_set_positions", "moa_kv_layout",
     "moa_workspace_bytes", "moa_workspace_init", "moa_workspace_check", "moa_prefill",
     "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws", "moa_stream_read", "moa_chunk_workspace_bytes",
-    "moa_prefill_chunk",
+    "moa_prefill_chunk", "moa_prefill_stall_test",
 )
 
 
@@ -69,6 +69,7 @@ def load():
         "moa_decode_append": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, P(i32), f32, vp, sz, vp]),
         "moa_decode_static_ws": (ctypes.c_int, [vp, vp, vp, i32, P(i32), f32, vp]),
         "moa_stream_read": (ctypes.c_int, [vp, sz, vp, vp]),
+        "moa_prefill_stall_test": (ctypes.c_int, [vp, vp, vp, vp, vp, sz, vp]),
         "moa_chunk_workspace_bytes": (ctypes.c_int, [vp, i32, i32, P(i32), P(sz)]),
         "moa_prefill_chunk": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, P(i32), f32, vp, sz, vp]),
     }
@@ -252,6 +253,12 @@ def moa_prefill_chunk(handle, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, str
     sp, spp = _i32(spans)
     _check(load().moa_prefill_chunk(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), Hq, n, spp, float(scale),
                                     _ptr(ws), int(ws_bytes), _stream(stream)), "moa_prefill_chunk")
+
+
+def moa_prefill_stall_test(q, k, v, o, ws, ws_bytes, stream=None):
+    """Launch the prefill kernel with its work units withheld (its bounded waits run out after 2 s)."""
+    _check(load().moa_prefill_stall_test(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), int(ws_bytes),
+                                         _stream(stream)), "moa_prefill_stall_test")
 
 
 def moa_stream_read(buf, nbytes, out, stream=None):

@@ -149,6 +149,20 @@ moa_status moa_workspace_init(void* workspace, size_t bytes, void* stream);
  * bounded wait in the last prefill using it gave up, else MOA_OK. */
 moa_status moa_workspace_check(const void* workspace, void* stream);
 
+/* Self-test of the failure path of the prefill kernel.  Every wait of the
+ * kernel on an mbarrier gives up after 2 s of wall time, records
+ * MOA_ERR_TIMEOUT in the workspace error word, lets the other roles leave,
+ * waits for its in-flight copies, frees its tensor memory and returns, so a
+ * lost arrival ends as a status instead of a hung GPU.  This call launches the
+ * kernel on a 1 x 1 x 128 x 128 bf16 problem (q, k, v, o: device, 16-byte
+ * aligned, 32 KB each) with its work-unit records withheld, so that path runs:
+ * after about 2 s moa_workspace_check(workspace) returns MOA_ERR_TIMEOUT and
+ * the context stays usable.  workspace: at least
+ * moa_workspace_bytes(MOA_OP_PREFILL, 1, 1, 128, 128, {128}) bytes, 256-byte
+ * aligned.  Not part of the attention path. */
+moa_status moa_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
 /* Read-only bandwidth probe for the decode roofline.  Decode attention
  * reads each head's window of K/V rows once per token and writes almost
  * nothing, so its bandwidth ceiling is a plain read stream.  Reads `bytes`

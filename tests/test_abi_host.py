@@ -203,6 +203,15 @@ def test_prefill_chunk_argument_errors_need_no_gpu():
     assert e.value.status == moa.MOA_ERR_INVALID_ARG
 
 
+def test_prefill_stall_test_argument_errors_need_no_gpu():
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_prefill_stall_test(None, 4096, 4096, 4096, 4096, 1 << 20, 0)
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    with pytest.raises(moa.MoaError) as e:          # workspace not 256-byte aligned
+        moa.moa_prefill_stall_test(4096, 4096, 4096, 4096, 4096 + 16, 1 << 20, 0)
+    assert e.value.status == moa.MOA_ERR_WORKSPACE
+
+
 def test_workspace_sizes():
     spans = [64, 300, 4096, 1]
     d = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)

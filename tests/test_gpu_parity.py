@@ -733,3 +733,29 @@ def test_bf16_decode_large_batch_sampled():
         hist_v = np.concatenate([vf[b], vnf[b]], axis=1)
         want = oatt.chunk(qf[b:b + 1, :, None, :], [hist_k], [hist_v], [prefix], spans, scale)[0, :, 0]
         assert np.max(np.abs(got[b] - want)) <= BF16_TOL, b
+
+
+def test_prefill_bounded_waits_report_a_timeout():
+    """Failure path without a fault: the prefill kernel launched with its work
+    units withheld gives up on its first waits after 2 s, the workspace error
+    word reads MOA_ERR_TIMEOUT, and a normal prefill on the same context still
+    matches the oracle."""
+    import time
+    d = 128
+    x = torch.zeros((1, 1, 128, d), dtype=torch.bfloat16, device=DEV)
+    o = torch.zeros_like(x)
+    ws = moa.Workspace(moa.MOA_OP_PREFILL, 1, 1, 128, d, [128])
+    torch.cuda.synchronize()
+    t0 = time.time()
+    moa.moa_prefill_stall_test(x, x, x, o, ws.ptr, ws.nbytes)
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_workspace_check(ws.ptr)
+    assert e.value.status == moa.MOA_ERR_TIMEOUT
+    assert 1.5 < time.time() - t0 < 60
+    spans = [200, 7]
+    q = inputs.randn(170, (1, 2, 300, d))
+    k = inputs.randn(171, (1, 1, 300, d))
+    v = inputs.randn(172, (1, 1, 300, d))
+    out = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, 1 / math.sqrt(d))
+    want = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, 1 / math.sqrt(d))
+    assert np.max(np.abs(inputs.as_f64(out) - want)) <= BF16_TOL
