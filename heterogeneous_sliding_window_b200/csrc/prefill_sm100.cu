@@ -860,7 +860,8 @@ namespace {
 moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, const void* kw,
                                     const void* vw, void* o, int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq,
                                     int32_t q_off, const int64_t* t, const int32_t* spans, float scale,
-                                    void* ws, size_t ws_bytes, cudaStream_t s, bool stall = false) {
+                                    void* ws, size_t ws_bytes, cudaStream_t s, bool stall = false,
+                                    const std::function<moa_status()>& before = nullptr) {
   if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
   const int32_t Nk = q_off + Nq;
@@ -886,8 +887,6 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   std::vector<int32_t> blob(kUnitsOffset / 4 + sch.units.size(), 0);
   std::copy(sch.off.begin(), sch.off.end(), blob.begin() + kOffsOffset / 4);
   std::copy(sch.units.begin(), sch.units.end(), blob.begin() + kUnitsOffset / 4);
-  cudaError_t e = cudaMemcpyAsync(ws, blob.data(), blob.size() * 4, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e, "prefill unit upload");
 
   PrefillParams p;
   p.hdr = reinterpret_cast<uint32_t*>(ws);
@@ -912,6 +911,15 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
   });
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "prefill smem attribute");
+  // All host work is done: whatever must run first on the stream (the chunk's
+  // window gather) goes in now, so the kernels follow one another without the
+  // device waiting on the host.
+  if (before) {
+    const moa_status st = before();
+    if (st != MOA_OK) return st;
+  }
+  const cudaError_t e = cudaMemcpyAsync(ws, blob.data(), blob.size() * 4, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill unit upload");
   prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mkw, mvw, p);
   return check_launch("prefill_bf16 launch");
 }
@@ -963,13 +971,12 @@ moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, c
   if (ws_bytes < L.bytes) return MOA_ERR_WORKSPACE;
   char* sk = static_cast<char*>(ws) + L.off_k;
   char* sv = static_cast<char*>(ws) + L.off_v;
-  moa_status st = MOA_OK;
-  if (L.W > 0) {
-    st = launch_gather_window(c, L.W, sk, sv, s);
-    if (st != MOA_OK) return st;
-  }
   const int64_t* t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
-  st = launch_prefill_bf16_rows(q, k, v, sk, sv, o, c->B, Hq, c->Hkv, n, L.W, t, spans, scale, ws, L.off_k, s);
+  const int32_t W = L.W;
+  moa_status st = launch_prefill_bf16_rows(q, k, v, sk, sv, o, c->B, Hq, c->Hkv, n, W, t, spans, scale, ws,
+                                           L.off_k, s, false, [&]() -> moa_status {
+                                             return W > 0 ? launch_gather_window(c, W, sk, sv, s) : MOA_OK;
+                                           });
   if (st != MOA_OK) return st;
   return launch_append(c, k, v, n, s);
 }
