@@ -43,7 +43,7 @@ typedef enum {
   MOA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or shape, NaN rule */
   MOA_ERR_CAPACITY = 2,     /* a span exceeds its key/value head's cache capacity  */
   MOA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moa_workspace_bytes */
-  MOA_ERR_UNSUPPORTED = 4,  /* valid request this build does not implement (e.g. bf16 d=64) */
+  MOA_ERR_UNSUPPORTED = 4,  /* valid request the library does not implement (e.g. bf16 d=64) */
   MOA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
   MOA_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (error word set) */
 } moa_status;

@@ -20,7 +20,7 @@ where g = h // (Hq // Hkv) is the key/value head that query head h reads
 (grouped-query attention; with Hq == Hkv, g == h).  Subtracting the row
 maximum leaves the result unchanged mathematically and keeps exp finite.
 
-Readings (listed in the design doc): the window holds S_h keys including the
+Readings taken where the pages are silent: the window holds S_h keys including the
 query's own position (S_h = 1 attends to itself only); no sink or global
 tokens; spans are per query head.
 

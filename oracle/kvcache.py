@@ -9,7 +9,7 @@ size.  The blog walkthrough (section 5) implements a static KV cache in its
 CUDA kernel.  A head with span S only ever reads its last S keys, so a
 cache of capacity C >= S that keeps the last C rows serves it exactly.
 
-Readings (listed in DESIGN.md):
+Readings taken where the pages are silent:
 
 * Spans are evaluated once, at the configured context length N, and stay
   fixed through decoding (the cache is static).

@@ -14,7 +14,7 @@ kernel's block-size requirement.  The worked example on the same page
 ("heads A, B, C" at N = 4k) shows head B with S = 5.6k and beta = 0 drawn as
 "100% of the input length" at 4k, so the span is clamped to N.
 
-Readings taken where the pages are silent (each listed in the design doc):
+Readings taken where the pages are silent:
 
 * Rounding to the block: nearest multiple of ``block``, ties rounded up,
   computed as ``block * floor(x / block + 0.5)`` in IEEE binary64 with every
