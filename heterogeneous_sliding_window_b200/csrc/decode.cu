@@ -584,15 +584,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
 // partial (m, l, o) per head is written or, with one split, o itself.
 constexpr int kMmaRows = 16;                      // cached rows per tile
 constexpr int kMmaTileBytes = kMmaRows * 128 * 2; // one 16 x 128 bf16 tile
+#ifndef MOA_MMA_STAGES
+#define MOA_MMA_STAGES 2
+#endif
+constexpr int kMmaStages = MOA_MMA_STAGES;        // K/V tiles in flight per warp + 1
+constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
 constexpr int kMmaWarpRows = kChunk / kDecWarps;  // entries per warp and split
-constexpr size_t kMmaSmem = (size_t)kDecWarps * (2 * 2 * kMmaTileBytes + 256);   // tiles + P scratch
+constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -672,9 +677,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     if (j == h1) e0b = W - Sh;
   }
 
-  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsm) + (uint32_t)warp * (2 * 2 * kMmaTileBytes + 256);
-  const uint32_t sP = sbase + 2 * 2 * kMmaTileBytes;             // [8 heads][16 rows] bf16
-  uint16_t* sPg = reinterpret_cast<uint16_t*>(dsm + (size_t)warp * (2 * 2 * kMmaTileBytes + 256) + 2 * 2 * kMmaTileBytes);
+  const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsm) + (uint32_t)warp * kMmaWarpBytes;
+  const uint32_t sP = sbase + kMmaStages * 2 * kMmaTileBytes;    // [8 heads][16 rows] bf16
+  uint16_t* sPg = reinterpret_cast<uint16_t*>(dsm + (size_t)warp * kMmaWarpBytes + kMmaStages * 2 * kMmaTileBytes);
   const int wrow0 = warp * kMmaWarpRows;                          // first split entry of this warp
   const int wrows = max(0, min(kMmaWarpRows, nrows - wrow0));
   const int ntiles = (wrows + kMmaRows - 1) / kMmaRows;
@@ -721,14 +726,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[mb][e] = 0.f;
 
-  if (ntiles > 0) load_tile(0, 0);
-  cp_async_commit();
-  for (int ti = 0; ti < ntiles; ++ti) {
-    if (ti + 1 < ntiles) load_tile(ti + 1, (ti + 1) & 1);
+  // prologue: the first kMmaStages - 1 tiles in flight (one commit group each)
+#pragma unroll
+  for (int k = 0; k < kMmaStages - 1; ++k) {
+    if (k < ntiles) load_tile(k, k);
     cp_async_commit();
-    cp_async_wait1();
+  }
+  for (int ti = 0; ti < ntiles; ++ti) {
+    const int nx = ti + kMmaStages - 1;
+    if (nx < ntiles) load_tile(nx, nx % kMmaStages);
+    cp_async_commit();
+    cp_async_wait<kMmaStages - 1>();                    // tile ti has landed
     __syncwarp();
-    const uint32_t tK = sbase + (uint32_t)(ti & 1) * 2 * kMmaTileBytes, tV = tK + kMmaTileBytes;
+    const uint32_t tK = sbase + (uint32_t)(ti % kMmaStages) * 2 * kMmaTileBytes, tV = tK + kMmaTileBytes;
     // S^T = K . Q^T
     float sacc[4] = {0.f, 0.f, 0.f, 0.f};
     {
@@ -790,7 +800,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     }
     __syncwarp();                                       // stage and scratch are rewritten next
   }
-  cp_async_wait0();
+  cp_async_wait<0>();
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, off);
