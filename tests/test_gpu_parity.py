@@ -759,3 +759,37 @@ def test_prefill_bounded_waits_report_a_timeout():
     out = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, 1 / math.sqrt(d))
     want = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, 1 / math.sqrt(d))
     assert np.max(np.abs(inputs.as_f64(out) - want)) <= BF16_TOL
+
+
+def test_bf16_decode_vicuna13b_mixed_layer_sampled():
+    """One layer of the 13B decode workload: B=8, 40 heads, context 16384, fixed-local
+    and elastic heads mixed to 50 % density, fused append; sampled heads against the
+    oracle's ring decode."""
+    B, H, d, N = 8, 40, 128, 16384
+    a, b = inputs.tables_13b_mix(9, H, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    cache = moa.KVCache(B, H, d, "bf16", spans)
+    data = cache.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(15, (data.numel(),)))
+    cache.set_positions([N] * B)
+    rng = np.random.default_rng(13)
+    picks = [(int(rng.integers(B)), int(rng.integers(H))) for _ in range(16)] + [(0, 0), (B - 1, H - 1)]
+    host = cache.data_bytes().cpu().numpy().tobytes()
+    blocks = {(bb, hh): okv.block_from_image(host, bb, hh, B, H, d, spans, "bf16") for bb, hh in picks}
+    scale = 1.0 / math.sqrt(d)
+    qt = inputs.randn_cuda(16, (B, H, d))
+    kt = inputs.randn_cuda(17, (B, H, 1, d))
+    vt = inputs.randn_cuda(18, (B, H, 1, d))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, spans)
+    ot = _nan_like((B, H, d), torch.bfloat16)
+    moa.moa_decode_append(cache.handle, qt, kt, vt, ot, H, spans, scale, ws.ptr, ws.nbytes)
+    torch.cuda.synchronize()
+    assert cache.positions() == [N + 1] * B
+    kt64, vt64, qt64, ot64 = (inputs.as_f64(x) for x in (kt, vt, qt, ot))
+    for bb, hh in picks:
+        K, V = blocks[(bb, hh)]
+        C = spans[hh]
+        K[N % C] = kt64[bb, hh, 0]
+        V[N % C] = vt64[bb, hh, 0]
+        ref = okv.decode_row_from_ring(K, V, N + 1, spans[hh], qt64[bb, hh], scale)
+        assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
