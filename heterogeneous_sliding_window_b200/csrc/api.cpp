@@ -2,6 +2,7 @@
 // Every check that can fail does so here, on the host, before anything is
 // enqueued; the kernels assume validated arguments.
 #include <algorithm>
+#include <mutex>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -17,6 +18,19 @@ int sm_count() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return 148;
   return n;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* done) {
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  std::lock_guard<std::mutex> lock(mu);
+  if (bit != 0 && (*done & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) *done |= bit;
+  return e;
 }
 
 moa_status cuda_fail(cudaError_t e, const char* where) {

@@ -891,8 +891,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
 
 template <int G>
 cudaError_t launch_group_mma(const DecodeParams& p, unsigned grid, cudaStream_t s) {
-  static cudaError_t attr = cudaFuncSetAttribute(decode_group_mma_kernel<G>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMmaSmem);
+  static unsigned long long attr_done = 0;
+  const cudaError_t attr =
+      ensure_smem_attr(reinterpret_cast<const void*>(decode_group_mma_kernel<G>), (int)kMmaSmem, &attr_done);
   if (attr != cudaSuccess) return attr;
   decode_group_mma_kernel<G><<<grid, kDecThreads, kMmaSmem, s>>>(p);
   return cudaGetLastError();

@@ -38,6 +38,11 @@ constexpr uint32_t kErrEmpty = 2u;
 
 int sm_count();
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute does not carry over between
+// devices); `done` is the caller's per-kernel record of devices already set.
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* done);
+
 // MOA_ERR_CUDA with the CUDA error reported on stderr when the environment
 // variable MOA_VERBOSE is set (the status alone cannot carry the reason).
 moa_status cuda_fail(cudaError_t e, const char* where);

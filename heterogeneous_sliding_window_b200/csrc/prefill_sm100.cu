@@ -904,12 +904,9 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.scale_log2 = scale * 1.4426950408889634f;
   for (int h = 0; h < Hq; ++h) p.span[h] = spans[h];
 
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(prefill_bf16_sm100_kernel,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-  });
+  static unsigned long long attr_done = 0;
+  const cudaError_t attr_err =
+      ensure_smem_attr(reinterpret_cast<const void*>(prefill_bf16_sm100_kernel), (int)SMEM_BYTES, &attr_done);
   if (attr_err != cudaSuccess) return cuda_fail(attr_err, "prefill smem attribute");
   // All host work is done: whatever must run first on the stream (the chunk's
   // window gather) goes in now, so the kernels follow one another without the
