@@ -270,16 +270,15 @@ def run_ours(args):
     kv_bytes_layer = [D_B * sum(2 * S * D_D * 2 for S in sp) + 2 * D_B * D_H * D_D * 2 + 4 * D_B * D_H * D_D * 2
                       for sp in d_spans]
     kv_bytes_step = sum(kv_bytes_layer)
-    launches_per_step = 2 + D_L
+    launches_per_step = 1 + D_L
 
     def step(ev):
         # rule evaluation for the prompt (host), prefill, cache fill, decode step
         moa.moa_rules_eval(pa, pb, P_N, BLOCK)
         ev["p0"].record(stream)
         moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", p_spans, p_scale, p_ws.ptr, p_ws.nbytes,
-                        None, stream)
+                        p_cache.handle, stream)       # the kernel also fills the prompt's cache
         ev["p1"].record(stream)
-        moa.moa_kv_append(p_cache.handle, k, v, P_N, stream)
         ev["d0"].record(stream)
         for layer in range(D_L):
             ev["k0"][layer].record(stream)
@@ -512,7 +511,7 @@ def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
                         "spans at 25% of 8192",
             "ms": round(ms, 4), "in_window_flops": int(flops), "tflops": round(tf, 2),
             "frac": round(tf / tf_peak, 4), "peak_kind": peak_kind + " burst (bf16_tflops)",
-            "launches": 3}
+            "launches": 2}
 
 
 def gqa_decode_layer(stream, reps=20):
@@ -612,10 +611,11 @@ def run_reference(args):
 def run_profile_case(case, launches=3):
     """Small single-kernel cases for ncu captures (a few GB on the device at most).
 
-    prefill: the 7B prompt (B=1, 32 heads, N=8192; Q/K/V 192 MiB), `launches` prefills.
+    prefill: the 7B prompt (B=1, 32 heads, N=8192; Q/K/V 192 MiB), `launches` prefills, each
+             filling the prompt's cache as the bench step does.
     decode : one decode layer of the 7B workload (B=32, 32 heads, context 4096; 1 GiB cache).
     chunk  : the bench's chunked prefill (4096-token chunk after 4096 cached tokens, 32 heads),
-             `launches` calls of moa_prefill_chunk (gather, prefill kernel, append each).
+             `launches` calls of moa_prefill_chunk (gather, then the prefill kernel with the append).
     gqa    : the bench's `gqa_decode` layer (Llama3-8B-shaped, B=32, 32/8 heads, context 8192,
              50 %; 0.96 GB of group windows), `launches` decode calls.
     """
@@ -630,10 +630,12 @@ def run_profile_case(case, launches=3):
         v = inputs.randn_cuda(12, (P_B, P_H, P_N, P_D))
         o = torch.empty_like(q)
         ws = moa.Workspace(moa.MOA_OP_PREFILL, P_B, P_H, P_N, P_D, sp)
+        pc = moa.KVCache(P_B, P_H, P_D, "bf16", sp)
         for _ in range(launches):
             moa.moa_prefill(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", sp, 1.0 / math.sqrt(P_D), ws.ptr,
-                            ws.nbytes)
+                            ws.nbytes, pc.handle)
         moa.moa_workspace_check(ws.ptr)
+        pc.positions()
     elif case == "gqa":
         B, Hq, Hkv, N, D = 32, 32, 8, 8192, 128
         a, b = inputs.tables_7b(1001, Hq, N, BLOCK, 0.5, moa.moa_rules_eval)

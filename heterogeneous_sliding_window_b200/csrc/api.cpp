@@ -245,7 +245,8 @@ extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, v
     if (d != 128) return MOA_ERR_UNSUPPORTED;
     if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
     if (ws_bytes < prefill_workspace_bytes(B, Hq, N)) return MOA_ERR_WORKSPACE;
-    st = launch_prefill_bf16(q, k, v, o, B, Hq, Hkv, (int32_t)N, spans, scale, ws, ws_bytes, s);
+    // the kernel writes the cache itself
+    return launch_prefill_bf16(q, k, v, o, B, Hq, Hkv, (int32_t)N, spans, scale, ws, ws_bytes, s, fill);
   }
   if (st != MOA_OK || !fill) return st;
   return launch_append(fill, k, v, (int32_t)N, s);

@@ -87,10 +87,12 @@ std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, con
                                            int32_t n_ctas);
 
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
+// fill != nullptr: the kernel also appends the N key/value rows to that cache
+// (the bytes and positions of launch_append(fill, k, v, N)).
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,
                                int32_t B, int32_t Hq, int32_t Hkv, int32_t N,
                                const int32_t* spans, float scale, void* ws, size_t ws_bytes,
-                               cudaStream_t s);
+                               cudaStream_t s, moa_kv_cache* fill = nullptr);
 
 // Self-test of the prefill kernel's bounded waits (prefill_sm100.cu): one CTA
 // on a 1 x 1 x 128 x 128 problem whose unit records are never published.

@@ -32,6 +32,9 @@
 //                   unit while tile B finishes this one.
 //      warp 2       unit fetcher: this CTA's unit records into a four-slot
 //                   ring in shared memory.
+//      warp 3       cache writer (when the call fills a KV cache): copies the
+//                   surviving key/value rows of its units into the ring
+//                   cache, so the fill needs no launch of its own.
 //      warps 4-7    softmax of tile A, warps 8-11 softmax of tile B: one
 //                   thread per query row reads its S row in two 64-column
 //                   halves, masks only tiles that cross the diagonal or the
@@ -52,8 +55,8 @@
 
 #include <algorithm>
 #include <functional>
+#include <memory>
 #include <mutex>
-#include <queue>
 
 #include "internal.h"
 #include "sm100.cuh"
@@ -65,7 +68,7 @@ using namespace sm100;
 
 constexpr int kThreads = 384;                    // 3 warpgroups
 // Register split (setmaxnreg): the block launches with 384 x 168 registers;
-// warpgroup 0 (producer, MMA issuer, unit fetcher, one idle warp) drops to
+// warpgroup 0 (producer, MMA issuer, unit fetcher, cache writer) drops to
 // 120, the two softmax warpgroups rise to 192.
 constexpr uint32_t kRegsLaunch = 168, kRegsControl = 120, kRegsSoftmax = 192;
 static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kThreads * kRegsLaunch, "register split");
@@ -131,7 +134,23 @@ struct PrefillParams {
   int32_t stall;                 // self-test of the bounded waits: the fetcher publishes nothing
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
+  // Cache fill (fill_data == nullptr: none).  Row r of k_rows / v_rows
+  // [B, Hkv, Nq, d] is position t_b + r of sequence b; the last min(Nq, C_g)
+  // rows go to ring slot (t_b + r) mod C_g of KV head g, and the last CTA to
+  // finish advances every t_b by Nq.
+  char* fill_data;               // cache data region
+  uint32_t* fill_ctr;            // cache header: completion counter
+  int64_t* fill_t;               // cache header: tokens per sequence
+  const char* k_rows;
+  const char* v_rows;
+  int64_t fill_sumC;             // sum of the capacities (row pairs per sequence)
+  int32_t B;
+  int32_t fill_cap[MOA_MAX_HEADS];
+  int64_t fill_goff[MOA_MAX_HEADS];
 };
+// The five tensor maps (128 bytes each) and the parameters share the 4 KB
+// kernel-parameter space.
+static_assert(sizeof(PrefillParams) + 5 * 128 <= 4096, "kernel parameters");
 
 struct Ctx {
   uint32_t bar0;                       // address of barrier 0
@@ -670,6 +689,61 @@ __device__ __forceinline__ void fetcher_role(const PrefillParams& p, const Ctx& 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Cache writer (warp 3, all lanes): for each unit of this CTA whose head is
+// the first of its KV group, copies the surviving key and value rows of the
+// unit's query tiles from k_rows / v_rows into the ring.  Each KV group's rows
+// are thus written exactly once.  The attention never reads the ring (its
+// keys come from k, v and the gathered window), so the copies need no
+// ordering with the other roles; only the position update waits for the
+// whole grid (see the end of the kernel).  Rows are 256 bytes (d = 128,
+// bf16): 16 lanes per row, two rows per load, eight rows per pass.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fill_role(const PrefillParams& p, int lane) {
+  constexpr int kRowBytes = kD * 2;
+  const int first = p.cta_off[blockIdx.x], last = p.cta_off[blockIdx.x + 1];
+  const int half = lane >> 4;                        // which of two rows
+  const size_t col = (size_t)(lane & 15) * 16;       // byte offset within the row
+  for (int u = first; u < last; ++u) {
+    const int4 U = p.units[u];
+    if (U.y % p.G != 0) continue;
+    const int g = U.y / p.G;
+    const int C = p.fill_cap[g];
+    const int q0 = U.z * 128 - p.q_off;              // the unit's first query row
+    const int r_first = max(q0, p.Nq - C);           // rows below Nq - C are overwritten later
+    const int r_end = min(q0 + 256, p.Nq);
+    if (r_first >= r_end) continue;
+    // r_end - r_first <= C, so slot0 + (r - r_first) wraps at most once
+    const int slot0 = (int)((p.fill_t[U.x] + r_first) % C);
+    char* kring = p.fill_data + (size_t)((int64_t)U.x * p.fill_sumC + p.fill_goff[g]) * 2 * kRowBytes;
+    char* vring = kring + (size_t)C * kRowBytes;
+    const size_t src0 = ((size_t)U.x * p.Hkv + g) * (size_t)p.Nq;
+    for (int r0 = r_first; r0 < r_end; r0 += 8) {
+      int4 kx[4], vx[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + 2 * j + half;
+        if (r < r_end) {
+          const size_t src = (src0 + r) * kRowBytes + col;
+          kx[j] = __ldg(reinterpret_cast<const int4*>(p.k_rows + src));
+          vx[j] = __ldg(reinterpret_cast<const int4*>(p.v_rows + src));
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = r0 + 2 * j + half;
+        if (r < r_end) {
+          int slot = slot0 + (r - r_first);
+          if (slot >= C) slot -= C;
+          const size_t dst = (size_t)slot * kRowBytes + col;
+          *reinterpret_cast<int4*>(kring + dst) = kx[j];
+          *reinterpret_cast<int4*>(vring + dst) = vx[j];
+        }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -723,6 +797,8 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       fetcher_role(p, c);
     else if (warp == 1 && lane == 0)
       mma_role(p, c, tmem, sbase + OFF_Q, sbase + OFF_K, sbase + OFF_V);
+    else if (warp == 3 && p.fill_data != nullptr)
+      fill_role(p, lane);
   } else {
     regs_inc<kRegsSoftmax>();
     softmax_role(p, c, tmem, warp < 8 ? 0 : 1, warp, lane);
@@ -738,6 +814,18 @@ prefill_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  // Cache fill: the last CTA to finish advances the positions.  Every CTA's
+  // fetcher and cache writer read t before the barrier above, so none of
+  // them can see the new value.
+  if (p.fill_data != nullptr && tid == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(p.fill_ctr, 1u);
+    if (prev == gridDim.x - 1) {
+      for (int b = 0; b < p.B; ++b) p.fill_t[b] += p.Nq;
+      *p.fill_ctr = 0u;
+      __threadfence();
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -786,42 +874,72 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
                                  int32_t m0) {
   const int64_t M = (N + kTileM - 1) / kTileM;      // key tiles; query tiles are m0 .. M-1
-  struct U { int32_t b, h, m, lo; int64_t cost; };
-  std::vector<U> v;
-  v.reserve((size_t)B * Hq * ((M - m0 + 1) / 2));
-  for (int32_t b = 0; b < B; ++b)
-    for (int32_t h = 0; h < Hq; ++h)
-      for (int64_t m = m0; m < M; m += 2) {
-        const int64_t lo = first_tile_host(m, spans[h]);
-        int64_t cost = m - lo + 1 + kUnitOverheadTiles;
-        if (m + 1 < M) cost += m + 1 - first_tile_host(m + 1, spans[h]) + 1;
-        v.push_back({b, h, (int32_t)m, (int32_t)lo, cost});
+  const int64_t per_head = std::max<int64_t>(0, (M - m0 + 1) / 2);
+  const int64_t n_units = (int64_t)B * Hq * per_head;
+  // unit u = (b * Hq + h) * per_head + k covers query tiles m0 + 2k and m0 + 2k + 1
+  std::vector<int32_t> lo((size_t)n_units), cost((size_t)n_units);
+  int32_t max_cost = 0;
+  for (int32_t h = 0; h < Hq; ++h)
+    for (int64_t k = 0; k < per_head; ++k) {
+      const int64_t m = m0 + 2 * k;
+      const int64_t l = first_tile_host(m, spans[h]);
+      int64_t c = m - l + 1 + kUnitOverheadTiles;
+      if (m + 1 < M) c += m + 1 - first_tile_host(m + 1, spans[h]) + 1;
+      for (int32_t b = 0; b < B; ++b) {
+        const size_t u = (size_t)(((int64_t)b * Hq + h) * per_head + k);
+        lo[u] = (int32_t)l;
+        cost[u] = (int32_t)c;
       }
-  std::stable_sort(v.begin(), v.end(), [](const U& a, const U& c) { return a.cost > c.cost; });
-  const int32_t n = (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_ctas, (int64_t)v.size()));
-  std::vector<std::vector<int32_t>> lists(n);
-  using Slot = std::pair<int64_t, int32_t>;          // (work so far, list)
-  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
-  for (int32_t c = 0; c < n; ++c) heap.push({0, c});
-  for (size_t i = 0; i < v.size(); ++i) {
-    Slot sl = heap.top();
-    heap.pop();
-    lists[sl.second].push_back((int32_t)i);
-    sl.first += v[i].cost;
-    heap.push(sl);
-  }
+      max_cost = std::max(max_cost, (int32_t)c);
+    }
+  // Longest first, equal costs in unit order: a stable counting sort.
+  std::vector<int32_t> start((size_t)max_cost + 2, 0);
+  for (int64_t u = 0; u < n_units; ++u) ++start[(size_t)(max_cost - cost[u]) + 1];
+  for (size_t i = 1; i < start.size(); ++i) start[i] += start[i - 1];
+  std::vector<int32_t> order((size_t)n_units);
+  for (int64_t u = 0; u < n_units; ++u) order[(size_t)start[(size_t)(max_cost - cost[u])]++] = (int32_t)u;
+  // Greedy LPT: each unit to the list with the least work so far (ties: the
+  // lowest list).  A binary min-heap of keys work * 2^11 + list: keys are
+  // distinct, so the minimum, and with it the schedule, does not depend on
+  // how the heap is arranged.  The chosen list's work only grows, so its key
+  // is sifted down from the root.
+  static_assert(kPrefillMaxCtas <= 2048, "list index field");
+  const int32_t n = (int32_t)std::max<int64_t>(1, std::min<int64_t>(n_ctas, n_units));
+  std::vector<uint64_t> heap((size_t)n);
+  for (int32_t c = 0; c < n; ++c) heap[(size_t)c] = (uint64_t)c;   // work 0, ascending lists: a heap
+  std::vector<int32_t> list_of((size_t)n_units);
   PrefillSchedule out;
   out.n_ctas = n;
-  out.off.assign(n + 1, 0);
-  out.units.reserve(v.size() * 4);
-  for (int32_t c = 0; c < n; ++c) {
-    for (int32_t i : lists[c]) {
-      out.units.push_back(v[i].b);
-      out.units.push_back(v[i].h);
-      out.units.push_back(v[i].m);
-      out.units.push_back(v[i].lo);
+  out.off.assign((size_t)n + 1, 0);
+  for (int64_t i = 0; i < n_units; ++i) {
+    const uint64_t top = heap[0];
+    const int32_t list = (int32_t)(top & 2047u);
+    list_of[(size_t)i] = list;
+    ++out.off[(size_t)list + 1];
+    const uint64_t key = top + ((uint64_t)cost[(size_t)order[(size_t)i]] << 11);
+    size_t pos = 0;
+    for (;;) {
+      size_t child = 2 * pos + 1;
+      if (child >= (size_t)n) break;
+      if (child + 1 < (size_t)n && heap[child + 1] < heap[child]) ++child;
+      if (heap[child] >= key) break;
+      heap[pos] = heap[child];
+      pos = child;
     }
-    out.off[c + 1] = (int32_t)(out.units.size() / 4);
+    heap[pos] = key;
+  }
+  for (int32_t c = 0; c < n; ++c) out.off[(size_t)c + 1] += out.off[(size_t)c];
+  // Each list in the order its units were dealt (longest first).
+  out.units.assign((size_t)n_units * 4, 0);
+  std::vector<int32_t> fill(out.off.begin(), out.off.end() - 1);
+  for (int64_t i = 0; i < n_units; ++i) {
+    const int32_t u = order[(size_t)i];
+    const int32_t bh = (int32_t)(u / per_head), k = (int32_t)(u % per_head);
+    int32_t* dst = &out.units[(size_t)fill[(size_t)list_of[(size_t)i]]++ * 4];
+    dst[0] = bh / Hq;
+    dst[1] = bh % Hq;
+    dst[2] = m0 + 2 * k;
+    dst[3] = lo[(size_t)u];
   }
   return out;
 }
@@ -852,6 +970,50 @@ size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
 
 namespace {
 
+// The workspace image of a schedule: zeroed header, per-CTA list offsets and
+// the units, uploaded in one copy.  The schedule depends only on the shapes,
+// the spans and the grid, so the last few images are kept and a call with the
+// same arguments (every layer of a model, every step of a server) reuses one
+// instead of rebuilding it.
+struct UnitBlob {
+  int32_t n_ctas = 0;
+  std::vector<int32_t> words;
+};
+
+struct BlobKey {
+  int32_t B, Hq, N, grid, m0;
+  std::vector<int32_t> spans;
+  bool operator==(const BlobKey& o) const {
+    return B == o.B && Hq == o.Hq && N == o.N && grid == o.grid && m0 == o.m0 && spans == o.spans;
+  }
+};
+
+std::shared_ptr<const UnitBlob> unit_blob(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t grid,
+                                          int32_t m0) {
+  constexpr size_t kKept = 8;
+  static std::mutex mu;
+  static std::vector<std::pair<BlobKey, std::shared_ptr<const UnitBlob>>> kept;   // most recent first
+  BlobKey key{B, Hq, N, grid, m0, std::vector<int32_t>(spans, spans + Hq)};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (size_t i = 0; i < kept.size(); ++i)
+      if (kept[i].first == key) {
+        std::rotate(kept.begin(), kept.begin() + (long)i, kept.begin() + (long)i + 1);
+        return kept[0].second;
+      }
+  }
+  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, grid, m0);
+  auto blob = std::make_shared<UnitBlob>();
+  blob->n_ctas = sch.n_ctas;
+  blob->words.assign(kUnitsOffset / 4 + sch.units.size(), 0);
+  std::copy(sch.off.begin(), sch.off.end(), blob->words.begin() + kOffsOffset / 4);
+  std::copy(sch.units.begin(), sch.units.end(), blob->words.begin() + kUnitsOffset / 4);
+  std::lock_guard<std::mutex> lock(mu);
+  kept.insert(kept.begin(), {std::move(key), blob});
+  if (kept.size() > kKept) kept.pop_back();
+  return blob;
+}
+
 // Query rows 0 .. Nq-1 are key positions q_off .. q_off+Nq-1 (q_off a
 // multiple of 128).  Key rows q_off .. q_off+Nq-1 are k, v [B, Hkv, Nq, d];
 // rows 0 .. q_off-1 are kw, vw [B, Hkv, q_off, d].  t: per-sequence token
@@ -860,7 +1022,8 @@ namespace {
 moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v, const void* kw,
                                     const void* vw, void* o, int32_t B, int32_t Hq, int32_t Hkv, int32_t Nq,
                                     int32_t q_off, const int64_t* t, const int32_t* spans, float scale,
-                                    void* ws, size_t ws_bytes, cudaStream_t s, bool stall = false,
+                                    void* ws, size_t ws_bytes, cudaStream_t s, moa_kv_cache* fill = nullptr,
+                                    bool stall = false,
                                     const std::function<moa_status()>& before = nullptr) {
   if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
@@ -883,10 +1046,8 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   const int64_t Mq = (Nq + kTileM - 1) / kTileM;
   const int64_t n_units = (int64_t)B * Hq * ((Mq + 1) / 2);
   const int32_t grid = (int32_t)std::min<int64_t>({n_units, (int64_t)sm_count(), (int64_t)kPrefillMaxCtas});
-  const PrefillSchedule sch = prefill_schedule(B, Hq, Nk, spans, grid, m0);
-  std::vector<int32_t> blob(kUnitsOffset / 4 + sch.units.size(), 0);
-  std::copy(sch.off.begin(), sch.off.end(), blob.begin() + kOffsOffset / 4);
-  std::copy(sch.units.begin(), sch.units.end(), blob.begin() + kUnitsOffset / 4);
+  const std::shared_ptr<const UnitBlob> sch = unit_blob(B, Hq, Nk, spans, grid, m0);
+  const std::vector<int32_t>& blob = sch->words;
 
   PrefillParams p;
   p.hdr = reinterpret_cast<uint32_t*>(ws);
@@ -903,6 +1064,24 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.G = Hq / Hkv;
   p.scale_log2 = scale * 1.4426950408889634f;
   for (int h = 0; h < Hq; ++h) p.span[h] = spans[h];
+  p.B = B;
+  p.fill_data = nullptr;
+  p.fill_ctr = nullptr;
+  p.fill_t = nullptr;
+  p.k_rows = static_cast<const char*>(k);
+  p.v_rows = static_cast<const char*>(v);
+  p.fill_sumC = 0;
+  if (fill != nullptr) {
+    if (fill->B != B || fill->Hkv != Hkv || fill->d != kD || fill->dtype != MOA_BF16) return MOA_ERR_INVALID_ARG;
+    p.fill_data = fill->buf + fill->header;
+    p.fill_ctr = reinterpret_cast<uint32_t*>(fill->buf + kHdrAppendCtr);
+    p.fill_t = reinterpret_cast<int64_t*>(fill->buf + kHdrT);
+    p.fill_sumC = fill->goff[Hkv];
+    for (int g = 0; g < Hkv; ++g) {
+      p.fill_cap[g] = fill->cap[g];
+      p.fill_goff[g] = fill->goff[g];
+    }
+  }
 
   static unsigned long long attr_done = 0;
   const cudaError_t attr_err =
@@ -917,7 +1096,7 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   }
   const cudaError_t e = cudaMemcpyAsync(ws, blob.data(), blob.size() * 4, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefill unit upload");
-  prefill_bf16_sm100_kernel<<<sch.n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mkw, mvw, p);
+  prefill_bf16_sm100_kernel<<<sch->n_ctas, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mkw, mvw, p);
   return check_launch("prefill_bf16 launch");
 }
 
@@ -945,16 +1124,16 @@ ChunkLayout chunk_layout(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const in
 
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
                                int32_t Hq, int32_t Hkv, int32_t N, const int32_t* spans, float scale,
-                               void* ws, size_t ws_bytes, cudaStream_t s) {
+                               void* ws, size_t ws_bytes, cudaStream_t s, moa_kv_cache* fill) {
   return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, B, Hq, Hkv, N, 0, nullptr, spans, scale, ws,
-                                  ws_bytes, s);
+                                  ws_bytes, s, fill);
 }
 
 moa_status launch_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* ws,
                                      size_t ws_bytes, cudaStream_t s) {
   const int32_t span = 128;
   return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, 1, 1, 1, 128, 0, nullptr, &span, 0.088f, ws,
-                                  ws_bytes, s, true);
+                                  ws_bytes, s, nullptr, true);
 }
 
 size_t prefill_chunk_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const int32_t* spans) {
@@ -970,12 +1149,12 @@ moa_status launch_prefill_chunk(moa_kv_cache* c, const void* q, const void* k, c
   char* sv = static_cast<char*>(ws) + L.off_v;
   const int64_t* t = reinterpret_cast<const int64_t*>(c->buf + kHdrT);
   const int32_t W = L.W;
-  moa_status st = launch_prefill_bf16_rows(q, k, v, sk, sv, o, c->B, Hq, c->Hkv, n, W, t, spans, scale, ws,
-                                           L.off_k, s, false, [&]() -> moa_status {
-                                             return W > 0 ? launch_gather_window(c, W, sk, sv, s) : MOA_OK;
-                                           });
-  if (st != MOA_OK) return st;
-  return launch_append(c, k, v, n, s);
+  // the prefill kernel also appends the chunk to the ring (its keys come from
+  // k, v and the gathered rows, never from the ring)
+  return launch_prefill_bf16_rows(q, k, v, sk, sv, o, c->B, Hq, c->Hkv, n, W, t, spans, scale, ws, L.off_k, s,
+                                  c, false, [&]() -> moa_status {
+                                    return W > 0 ? launch_gather_window(c, W, sk, sv, s) : MOA_OK;
+                                  });
 }
 
 }  // namespace moa

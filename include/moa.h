@@ -185,8 +185,10 @@ moa_status moa_stream_read(const void* buf, size_t bytes, void* out, void* strea
  * bytes; MOA_F32 may pass workspace NULL.  The schedule of work units is
  * uploaded into the workspace from host memory on every call.
  * fill_or_null: if non-NULL, a cache with B, Hkv, d and dtype equal to this
- * call's, spans[h] <= C_{h/(Hq/Hkv)}; after attention the prompt's K/V are
- * appended to it exactly as moa_kv_append(cache, k, v, N) would.
+ * call's, spans[h] <= C_{h/(Hq/Hkv)}; the prompt's K/V are appended to it
+ * exactly as moa_kv_append(cache, k, v, N) would (same bytes and positions).
+ * MOA_BF16 writes the cache inside the prefill kernel (one launch in all);
+ * MOA_F32 appends with a second launch.
  * ------------------------------------------------------------------------- */
 moa_status moa_prefill(const void* q, const void* k, const void* v, void* o,
                        int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
@@ -227,10 +229,11 @@ moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t*
  *   initialisation needed; it holds the work-unit schedule and the window's
  *   key/value rows gathered from the ring, [B, Hkv, W, d] with
  *   W = max_h S_h - 1 rounded up to 128.
- * Three launches on `stream` (two when every span is 1): the window gather,
- * the tensor-core prefill kernel (key tiles below W from the gathered rows,
- * the chunk's own straight from k, v; rows of negative positions masked),
- * the append.  Errors as moa_prefill. */
+ * Two launches on `stream` (one when every span is 1): the window gather,
+ * then the tensor-core prefill kernel (key tiles below W from the gathered
+ * rows, the chunk's own straight from k, v; rows of negative positions
+ * masked), which also appends the chunk to the ring.  Errors as
+ * moa_prefill. */
 moa_status moa_chunk_workspace_bytes(const moa_kv_cache* cache, int32_t Hq, int32_t n,
                                      const int32_t* spans, size_t* bytes_out);
 moa_status moa_prefill_chunk(moa_kv_cache* cache, const void* q, const void* k, const void* v,

@@ -141,6 +141,39 @@ def test_bf16_prefill_fill_cache_bytes():
     assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "bf16")
 
 
+def test_bf16_prefill_fill_after_cached_tokens():
+    """The prefill kernel's cache writer appends after tokens already held:
+    per-sequence positions differ, the ring wraps inside a prompt, MHA and
+    GQA, a prompt longer than some capacities.  Bytes and positions equal the
+    ring emulation's, and the attention output is unchanged by the fill."""
+    for (B, Hq, Hkv, N, spans, t0) in [(2, 3, 3, 700, [64, 300, 700], [0, 0]),
+                                       (2, 4, 2, 333, [129, 64, 256, 200], [5, 300]),
+                                       (3, 2, 1, 128, [1, 128], [7, 0, 1000])]:
+        d = 128
+        caps = okv.group_capacities(spans, Hkv)
+        seed = 40 + N
+        k0 = inputs.randn(seed, (B, Hkv, max(t0) or 1, d))
+        v0 = inputs.randn(seed + 1, (B, Hkv, max(t0) or 1, d))
+        q = inputs.randn(seed + 2, (B, Hq, N, d))
+        k = inputs.randn(seed + 3, (B, Hkv, N, d))
+        v = inputs.randn(seed + 4, (B, Hkv, N, d))
+        cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+        ring = okv.RingCache(B, Hkv, d, caps)
+        # history of t0[b] tokens per sequence: append per sequence length by
+        # filling all, then setting the positions the emulation reaches
+        if max(t0) > 0:
+            moa.moa_kv_append(cache.handle, k0.to(DEV), v0.to(DEV), max(t0))
+            ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+            cache.set_positions(t0)
+            ring.t = list(t0)
+        o = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, 0.1, fill=cache)
+        ring.append(inputs.as_f64(k), inputs.as_f64(v))
+        assert cache.positions() == [t + N for t in t0]
+        assert bytes(cache.data_bytes().cpu().numpy()) == okv.data_image(ring, "bf16")
+        ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, 0.1)
+        assert np.max(np.abs(inputs.as_f64(o) - ref)) <= BF16_TOL
+
+
 def _sample_rows(B, H, N, rng, n=96):
     rows = set()
     for b in range(B):
