@@ -393,6 +393,8 @@ def run_ours(args):
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
     chunk = chunk_prefill(stream, tf_peak, peak_kind)
+    p_alone_ms = prefill_alone(stream, q, k, v, o, p_spans, p_scale, p_ws, p_cache)
+    p_alone_tf = p_flops / (p_alone_ms * 1e-3) / 1e12
     read_gbs = read_only_gbs([c.data_bytes() for c in caches[:4]], stream)
 
     result = None
@@ -425,7 +427,11 @@ def run_ours(args):
                                      "peak_kind": peak_kind + " burst (bf16_tflops)",
                                      "frac_of_sustained": round(p_achieved / tf_sustained, 4),
                                      "frac_of_nominal": round(p_achieved / NOMINAL_BF16_TFLOPS, 4),
-                                     "traffic": traffic.get("prefill")}},
+                                     "traffic": traffic.get("prefill")},
+                        "alone": {"ms": round(p_alone_ms, 4), "tflops": round(p_alone_tf, 2),
+                                  "frac": round(p_alone_tf / tf_peak, 4),
+                                  "note": "the same call (prefill + cache fill) back to back, outside the step; "
+                                          "192 MiB of Q/K/V per call"}},
             "e2e": {"value": round(job_throughput(D_B, ws_n, e2e_ms), 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "note": "decode step through the C ABI from pinned host q/k/v to host o; copies on a "
@@ -465,6 +471,29 @@ def read_only_gbs(bufs, stream, reps=5):
         torch.cuda.synchronize()
         best = min(best, e0.elapsed_time(e1))
     return sum(sizes) / (best * 1e-3) / 1e9
+
+
+def prefill_alone(stream, q, k, v, o, spans, scale, ws, cache, reps=20):
+    """The bench step's prefill call (attention + the prompt's cache fill) timed back to back
+    outside the step: mean ms per call over `reps` calls after 3 untimed ones."""
+    import torch
+    from heterogeneous_sliding_window_b200 import moa
+    B, H, N, D = q.shape
+
+    def call():
+        moa.moa_prefill(q, k, v, o, B, H, H, N, D, "bf16", spans, scale, ws.ptr, ws.nbytes, cache.handle, stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    moa.moa_workspace_check(ws.ptr)
+    return e0.elapsed_time(e1) / reps
 
 
 def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
