@@ -262,11 +262,17 @@ __device__ __forceinline__ void load_half(uint32_t tS, int hh, int hi_c, int lo_
 #pragma unroll
   for (int cc = 0; cc < 64; ++cc) s[cc] = __uint_as_float(sr[cc]);
   if (edge) {
+    // Keep the columns lo_c < col <= hi_c: bits a..b of a 64-bit word built
+    // once per half, so each score costs one bit test and one select rather
+    // than two compares and a select (integer compares and selects issue at
+    // half the rate of the FMA pipe).
+    const int a = max(lo_c + 1 - 64 * hh, 0), b = min(hi_c - 64 * hh, 63);
+    const unsigned long long keep =
+        a > b ? 0ull : ((~0ull) >> (63 - max(b, 0))) & ((~0ull) << min(a, 63));
+    const uint32_t k0 = (uint32_t)keep, k1 = (uint32_t)(keep >> 32);
 #pragma unroll
-    for (int cc = 0; cc < 64; ++cc) {
-      const int col = 64 * hh + cc;
-      if (col > hi_c || col <= lo_c) s[cc] = -INFINITY;
-    }
+    for (int cc = 0; cc < 64; ++cc)
+      if (!(((cc < 32 ? k0 : k1) >> (cc & 31)) & 1u)) s[cc] = -INFINITY;
   }
 }
 
