@@ -148,7 +148,9 @@ def test_bf16_prefill_fill_after_cached_tokens():
     ring emulation's, and the attention output is unchanged by the fill."""
     for (B, Hq, Hkv, N, spans, t0) in [(2, 3, 3, 700, [64, 300, 700], [0, 0]),
                                        (2, 4, 2, 333, [129, 64, 256, 200], [5, 300]),
-                                       (3, 2, 1, 128, [1, 128], [7, 0, 1000])]:
+                                       (3, 2, 1, 128, [1, 128], [7, 0, 1000]),
+                                       (1, 2, 2, 5, [1, 5], [3]),
+                                       (2, 1, 1, 1, [1], [0, 9])]:
         d = 128
         caps = okv.group_capacities(spans, Hkv)
         seed = 40 + N
@@ -159,8 +161,9 @@ def test_bf16_prefill_fill_after_cached_tokens():
         v = inputs.randn(seed + 4, (B, Hkv, N, d))
         cache = moa.KVCache(B, Hkv, d, "bf16", caps)
         ring = okv.RingCache(B, Hkv, d, caps)
-        # history of t0[b] tokens per sequence: append per sequence length by
-        # filling all, then setting the positions the emulation reaches
+        # a history: max(t0) tokens appended to every sequence, then each
+        # sequence's position set to t0[b] (the ring bytes stay, only the
+        # positions move), in the emulation as well
         if max(t0) > 0:
             moa.moa_kv_append(cache.handle, k0.to(DEV), v0.to(DEV), max(t0))
             ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
