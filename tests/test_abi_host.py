@@ -135,6 +135,49 @@ def test_prefill_schedule_covers_band(N, spans, n_ctas):
     assert max(totals) - min(totals) <= max(cost.values())
 
 
+def _greedy_lpt(B, Hq, N, spans, n_ctas):
+    """The schedule rule in plain Python: units of query tiles (m, m+1) of one
+    (b, h), cost = their key-tile count + 4, sorted by cost (longest first,
+    ties in (b, h, m) order), each dealt to the list with the least work
+    (ties: the lowest list).  Returns the rows moa_prefill_schedule reports."""
+    M = (N + 127) // 128
+    first = lambda t, S: max(0, 128 * t - S + 1) // 128     # noqa: E731
+    units = []
+    for b in range(B):
+        for h in range(Hq):
+            for m in range(0, M, 2):
+                cost = m - first(m, spans[h]) + 1 + 4
+                if m + 1 < M:
+                    cost += m + 1 - first(m + 1, spans[h]) + 1
+                units.append((cost, b, h, m))
+    order = sorted(range(len(units)), key=lambda i: -units[i][0])   # Python's sort is stable
+    n = max(1, min(n_ctas, len(units)))
+    work = [0] * n
+    lists = [[] for _ in range(n)]
+    for i in order:
+        c = min(range(n), key=lambda j: (work[j], j))
+        lists[c].append(i)
+        work[c] += units[i][0]
+    rows, k = [], 0
+    for c in range(n):
+        for i in lists[c]:
+            _, b, h, m = units[i]
+            for t in range(m, min(m + 2, M)):
+                rows.append((c, k, b, h, t, first(t, spans[h]), t))
+            k += 1
+    return rows
+
+
+@pytest.mark.parametrize("B,N,spans,n_ctas", [(1, 8192, None, 148), (2, 1000, [1, 64, 300, 1000, 129], 7),
+                                              (3, 640, [256, 700], 5), (1, 129, [2, 129], 148)])
+def test_prefill_schedule_is_the_greedy_lpt_rule(B, N, spans, n_ctas):
+    if spans is None:                        # the bench prompt's spans
+        a, b = inputs.tables_7b(1, 32, N, 64, 0.25, orules.eval_spans)
+        spans = orules.eval_spans(a, b, N, 64)
+    got = [tuple(r) for r in moa.moa_prefill_schedule(B, len(spans), N, spans, n_ctas).tolist()]
+    assert got == _greedy_lpt(B, len(spans), N, spans, n_ctas)
+
+
 def test_prefill_schedule_arguments():
     with pytest.raises(moa.MoaError):
         moa.moa_prefill_schedule(1, 1, 128, [64], 0)
