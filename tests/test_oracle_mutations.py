@@ -51,6 +51,8 @@ def test_pins_pass_on_the_oracle_as_written():
     assert not _fails(ATT.test_chunk_equals_prefill_rows_of_the_whole_sequence)
     assert not _fails(KV.test_layout_sizes_and_offsets)
     assert not _fails(KV.test_decode_equals_last_prefill_row)
+    assert not _fails(KV.test_ring_holds_last_capacity_tokens)
+    assert not _fails(ATT.test_in_window_flops_counts_mask_entries)
 
 
 def test_window_one_key_too_wide_is_caught(monkeypatch):
@@ -164,3 +166,39 @@ def test_span_without_the_clamp_is_caught(monkeypatch):
     monkeypatch.setattr(rules, "span_rule", _span_variant(lambda y: math.floor(y + 0.5), clamp=False))
     assert _fails(RULES.test_clamps)
     assert any(_fails(RULES.test_project_page_worked_heads, row) for row in RULES._golden_rows())
+
+
+def test_ring_keeping_the_first_rows_of_a_long_append_is_caught(monkeypatch):
+    def append(self, k, v):
+        k = np.asarray(k, dtype=np.float64)
+        v = np.asarray(v, dtype=np.float64)
+        B, Hkv, n, d = k.shape
+        for b in range(B):
+            for g in range(Hkv):
+                C = self.C[g]
+                for r in range(min(n, C)):                           # the first C rows, not the last
+                    s = self.slot(self.t[b] + r, C)
+                    self.K[b][g][s] = k[b, g, r]
+                    self.V[b][g][s] = v[b, g, r]
+                    self.written[b][g][s] = True
+            self.t[b] += n
+    monkeypatch.setattr(kvcache.RingCache, "append", append)
+    assert _fails(KV.test_ring_holds_last_capacity_tokens)
+
+
+def test_ring_not_advancing_positions_is_caught(monkeypatch):
+    orig = kvcache.RingCache.append
+
+    def append(self, k, v):
+        t = list(self.t)
+        orig(self, k, v)
+        self.t = t                                                   # t_b += n dropped
+    monkeypatch.setattr(kvcache.RingCache, "append", append)
+    assert _fails(KV.test_ring_holds_last_capacity_tokens)
+
+
+def test_flops_without_the_causal_triangle_is_caught(monkeypatch):
+    def in_window_flops(spans, N, d, B=1):
+        return B * sum(4 * d * min(int(S), int(N)) * N for S in spans)   # dropped S(S-1)/2 term
+    monkeypatch.setattr(attention, "in_window_flops", in_window_flops)
+    assert _fails(ATT.test_in_window_flops_counts_mask_entries)
