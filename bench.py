@@ -43,6 +43,12 @@ NOMINAL_BF16_TFLOPS = 2250.0
 P_B, P_H, P_N, P_D, P_DENSITY, P_SEED = 1, 32, 8192, 128, 0.25, 1
 D_L, D_B, D_H, D_N, D_D, D_DENSITY, D_SEED = 32, 32, 32, 4096, 128, 0.5, 1000
 BLOCK = 64
+# Vicuna-13B-shaped prefill + decode: 40 layers x 40 heads, d=128, N=16384, 50% density mixing
+# fixed-local and elastic heads; decode batch 8 for 128 steps
+V13_L, V13_H, V13_N, V13_D, V13_DENSITY, V13_B, V13_STEPS, V13_SEED = 40, 40, 16384, 128, 0.5, 8, 128, 3000
+# Llama3-8B-shaped GQA prefill: 32 query heads on 8 KV heads, d=128, N=32768, B=1, density sweep
+L3_HQ, L3_HKV, L3_N, L3_D, L3_SEED = 32, 8, 32768, 128, 4000
+L3_DENSITIES = (0.125, 0.25, 0.5, 1.0)
 
 
 def _peaks():
@@ -118,6 +124,78 @@ class Clocks:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+class ClockSampler:
+    """Read-only clock record of one timed region: a thread polls NVML's SM clock and
+    clocks-event (throttle) reasons every `period` seconds while the region runs.
+
+    Nothing is set: only NVML queries.  Falls back to the nvidia-smi sampler when NVML
+    cannot be opened.
+    """
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, uuid=None, index=0, period=0.002):
+        self.period = period
+        self.handle = None
+        self.fallback = None
+        self.thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid
+                           else pynvml.nvmlDeviceGetHandleByIndex(index))
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+            self.fallback = Clocks(uuid if uuid else index)
+
+    @staticmethod
+    def for_current_device(period=0.002):
+        import torch
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+        except Exception:
+            uuid = None
+        return ClockSampler(uuid, torch.cuda.current_device(), period)
+
+    def start(self):
+        if self.handle is None:
+            self.fallback.start()
+            return
+        import threading
+        self.sm, self.bits = [], 0
+        self.stop_ev = threading.Event()
+
+        def poll():
+            nv, h = self.nv, self.handle
+            while not self.stop_ev.is_set():
+                try:
+                    self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    self.bits |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                except Exception:
+                    pass
+                self.stop_ev.wait(self.period)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.handle is None:
+            return self.fallback.stop()
+        self.stop_ev.set()
+        self.thread.join()
+        if not self.sm:
+            return None
+        reasons = [name for name, attr in self.REASONS if self.bits & int(getattr(self.nv, attr, 0))]
+        return {"sm_mhz": statistics.median(self.sm), "sm_min_mhz": min(self.sm), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.sm), "source": "nvml poll %.0f ms" % (1e3 * self.period)}
 
 
 def _dist():
@@ -214,6 +292,52 @@ def oracle_prefill_sample(seconds_budget=10.0):
     return flops / timed / 1e9, "%d query rows (every 97th row x every 4th head) of the prompt" % n
 
 
+def oracle_prefill_rate(spans, N, d, seconds_budget=5.0, stride=97, seed=9):
+    """Oracle in-window GFLOP/s on a bounded sample of query rows (every `stride`-th row from the
+    end, every 4th head) of a prompt with these per-head spans."""
+    from oracle import attention as oatt
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    scale = 1.0 / math.sqrt(d)
+    timed, flops, n = 0.0, 0, 0
+    for i in range(N - 1, 0, -stride):
+        for h in range(0, len(spans), 4):
+            lo = max(0, i - spans[h] + 1)
+            q = rng.standard_normal(d)
+            t0 = time.perf_counter()
+            oatt.attend_row(q, K, V, lo, i, scale)
+            timed += time.perf_counter() - t0
+            flops += 4 * d * (i - lo + 1)
+            n += 1
+        if timed > seconds_budget:
+            break
+    return flops / timed / 1e9, n
+
+
+def oracle_decode_rate(spans, d, seqs=2, seed=10):
+    """Oracle seconds for one decode token of one layer: `seqs` sequences x every head of the
+    layer over fresh N(0,1) windows, per sequence."""
+    from oracle import attention as oatt
+    rng = np.random.default_rng(seed)
+    scale = 1.0 / math.sqrt(d)
+    timed = 0.0
+    for _ in range(seqs):
+        for S in spans:
+            K = rng.standard_normal((S, d))
+            V = rng.standard_normal((S, d))
+            q = rng.standard_normal(d)
+            t0 = time.perf_counter()
+            oatt.attend_row(q, K, V, 0, S - 1, scale)
+            timed += time.perf_counter() - t0
+    return timed / seqs
+
+
+def prefill_flops(spans, N, d, B=1):
+    """In-window FLOPs of a prompt: 4 d sum_h (S N - S (S - 1) / 2), S = min(S_h, N)."""
+    return B * sum(4 * d * (min(S, N) * N - min(S, N) * (min(S, N) - 1) // 2) for S in spans)
+
+
 # ---------------------------------------------------------------------------
 # GPU path
 # ---------------------------------------------------------------------------
@@ -297,10 +421,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     moa.moa_workspace_check(p_ws.ptr)
 
-    try:
-        clocks = Clocks("GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid))
-    except Exception:
-        clocks = Clocks(torch.cuda.current_device())
+    clocks = ClockSampler.for_current_device()
     evs = [new_events() for _ in range(args.steps)]
     if dist:
         dist.barrier()
@@ -393,9 +514,15 @@ def run_ours(args):
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
     chunk = chunk_prefill(stream, tf_peak, peak_kind)
-    p_alone_ms = prefill_alone(stream, q, k, v, o, p_spans, p_scale, p_ws, p_cache)
+    p_alone_ms, p_alone_clk = prefill_alone(stream, q, k, v, o, p_spans, p_scale, p_ws, p_cache)
     p_alone_tf = p_flops / (p_alone_ms * 1e-3) / 1e12
     read_gbs = read_only_gbs([c.data_bytes() for c in caches[:4]], stream)
+    # the other workloads: free the 7B decode state first (34 GB of caches)
+    del caches, d_ws, d_q, d_k, d_v, d_o, e_q, e_k, e_v
+    torch.cuda.empty_cache()
+    peaks = (hbm_peak, tf_peak, tf_sustained, peak_kind)
+    v13 = vicuna13b(stream, peaks, read_gbs, args.cpu_seconds, rank == 0) if not args.skip_extra else None
+    l3 = llama3_gqa_prefill(stream, peaks, args.cpu_seconds, rank == 0) if not args.skip_extra else None
 
     result = None
     if rank == 0:
@@ -429,7 +556,7 @@ def run_ours(args):
                                      "frac_of_nominal": round(p_achieved / NOMINAL_BF16_TFLOPS, 4),
                                      "traffic": traffic.get("prefill")},
                         "alone": {"ms": round(p_alone_ms, 4), "tflops": round(p_alone_tf, 2),
-                                  "frac": round(p_alone_tf / tf_peak, 4),
+                                  "frac": round(p_alone_tf / tf_peak, 4), "clocks": p_alone_clk,
                                   "note": "the same call (prefill + cache fill) back to back, outside the step; "
                                           "192 MiB of Q/K/V per call"}},
             "e2e": {"value": round(job_throughput(D_B, ws_n, e2e_ms), 2), "unit": "tokens/s",
@@ -438,6 +565,8 @@ def run_ours(args):
                             "second stream overlap the kernels"},
             "gqa_decode": gqa,
             "prefill_chunk": chunk,
+            "vicuna13b": v13,
+            "llama3_gqa_prefill": l3,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clock_info,
             "cpu_baseline": {"value": round(cpu_tok, 4), "unit": "tokens/s", "cores": _oracle_threads(),
@@ -473,30 +602,39 @@ def read_only_gbs(bufs, stream, reps=5):
     return sum(sizes) / (best * 1e-3) / 1e9
 
 
-def prefill_alone(stream, q, k, v, o, spans, scale, ws, cache, reps=20):
-    """The bench step's prefill call (attention + the prompt's cache fill) timed back to back
-    outside the step: mean ms per call over `reps` calls after 3 untimed ones."""
+def back_to_back(stream, call, reps, warmup=3):
+    """Mean ms per call of `reps` back-to-back calls on `stream` (CUDA events), after `warmup`
+    untimed ones, with the clock record of the timed region."""
     import torch
-    from heterogeneous_sliding_window_b200 import moa
-    B, H, N, D = q.shape
-
-    def call():
-        moa.moa_prefill(q, k, v, o, B, H, H, N, D, "bf16", spans, scale, ws.ptr, ws.nbytes, cache.handle, stream)
-    for _ in range(3):
+    for _ in range(warmup):
         call()
     torch.cuda.synchronize()
+    clocks = ClockSampler.for_current_device()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    clocks.start()
     e0.record(stream)
     for _ in range(reps):
         call()
     e1.record(stream)
     torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps, clocks.stop()
+
+
+def prefill_alone(stream, q, k, v, o, spans, scale, ws, cache, reps=200):
+    """The bench step's prefill call (attention + the prompt's cache fill) timed back to back
+    outside the step: mean ms per call over `reps` calls after 3 untimed ones, and the clocks."""
+    from heterogeneous_sliding_window_b200 import moa
+    B, H, N, D = q.shape
+
+    def call():
+        moa.moa_prefill(q, k, v, o, B, H, H, N, D, "bf16", spans, scale, ws.ptr, ws.nbytes, cache.handle, stream)
+    ms, clk = back_to_back(stream, call, reps)
     moa.moa_workspace_check(ws.ptr)
-    return e0.elapsed_time(e1) / reps
+    return ms, clk
 
 
-def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
+def chunk_prefill(stream, tf_peak, peak_kind, reps=40):
     """Chunked prefill into the ring cache: a Vicuna-7B-shaped layer (32 heads,
     d=128, spans at 25 % of 8192) holds the first 4096 tokens of a prompt and
     takes the other 4096 in one moa_prefill_chunk call (window gather,
@@ -524,7 +662,10 @@ def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
     moa.moa_prefill_chunk(cache.handle, q0, k0, v0, o0, H, t, spans, scale, wptr, nb, stream)
     flops = sum(4 * d * sum(min(t + i + 1, S) for i in range(n)) for S in spans) * B
     times = []
+    clocks = ClockSampler.for_current_device()
     for r in range(reps + 3):
+        if r == 3:
+            clocks.start()
         cache.set_positions([t], stream)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -534,16 +675,17 @@ def chunk_prefill(stream, tf_peak, peak_kind, reps=10):
         torch.cuda.synchronize()
         if r >= 3:
             times.append(e0.elapsed_time(e1))
+    clk = clocks.stop()
     ms = statistics.median(times)
     tf = flops / (ms * 1e-3) / 1e12
     return {"workload": "vicuna7b-shaped layer: 4096-token chunk after 4096 cached tokens, H=32 d=128, "
                         "spans at 25% of 8192",
             "ms": round(ms, 4), "in_window_flops": int(flops), "tflops": round(tf, 2),
             "frac": round(tf / tf_peak, 4), "peak_kind": peak_kind + " burst (bf16_tflops)",
-            "launches": 2}
+            "launches": 2, "clocks": clk}
 
 
-def gqa_decode_layer(stream, reps=20):
+def gqa_decode_layer(stream, reps=300):
     """One Llama3-8B-shaped grouped-query decode layer (B=32, 32 query heads on 8 KV heads,
     d=128, context 8192, per-head spans at 50% density), timed back to back with CUDA events.
 
@@ -565,18 +707,9 @@ def gqa_decode_layer(stream, reps=20):
     q = inputs.randn_cuda(2001, (B, Hq, D))
     o = torch.empty_like(q)
     scale = 1.0 / math.sqrt(D)
-    for _ in range(3):
-        moa.moa_decode(c.handle, q, o, Hq, sp, scale, ws.ptr, ws.nbytes, stream)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        moa.moa_decode(c.handle, q, o, Hq, sp, scale, ws.ptr, ws.nbytes, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    ms, clk = back_to_back(stream, lambda: moa.moa_decode(c.handle, q, o, Hq, sp, scale, ws.ptr, ws.nbytes, stream),
+                           reps)
     c.positions()
-    ms = e0.elapsed_time(e1) / reps
     group_bytes = B * sum(2 * cp * D * 2 for cp in caps) + 2 * B * Hq * D * 2
     head_bytes = B * sum(2 * S * D * 2 for S in sp) + 2 * B * Hq * D * 2
     c.close()
@@ -586,7 +719,193 @@ def gqa_decode_layer(stream, reps=20):
             "frac_of_copy": round(group_bytes / (ms * 1e-3) / 1e9 / _peaks()[0], 4),
             "ms": round(ms, 4), "group_window_bytes": group_bytes, "per_head_window_bytes": head_bytes,
             "gbs_of_group_bytes": round(group_bytes / (ms * 1e-3) / 1e9, 1),
-            "tokens_per_s_one_layer": round(B / (ms * 1e-3), 1)}
+            "tokens_per_s_one_layer": round(B / (ms * 1e-3), 1), "clocks": clk}
+
+
+def vicuna13b(stream, peaks, read_gbs, cpu_seconds, with_cpu):
+    """Vicuna-13B-shaped prefill + decode, each timed in its own clock-sampled region.
+
+    Prefill: 40 layers, each with its own fixed-local/elastic span mix at 50 % of N=16384 and
+    its prompt's cache fill; one Q/K/V set (480 MiB, larger than L2) serves every layer.
+    Decode: 40 layers x 40 heads, B=8, context 16384, caches prefilled with N(0,1) (53.7 GB),
+    V13_STEPS steps of 40 fused append+decode launches.
+    """
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    hbm_peak, tf_peak, tf_sustained, peak_kind = peaks
+    L, H, N, D, B = V13_L, V13_H, V13_N, V13_D, V13_B
+    scale = 1.0 / math.sqrt(D)
+    spans = []
+    for layer in range(L):
+        a, b = inputs.tables_13b_mix(V13_SEED + layer, H, N, BLOCK, V13_DENSITY, moa.moa_rules_eval)
+        spans.append(moa.moa_rules_eval(a, b, N, BLOCK))
+    out = {"workload": "vicuna13b-shaped: %d layers x %d heads, d=%d, N=%d, density %.2f (fixed-local alpha in "
+                       "{1024,2048} and elastic beta in {0.5,0.9} heads); decode B=%d for %d steps"
+                       % (L, H, D, N, V13_DENSITY, B, V13_STEPS),
+           "mean_density": round(float(np.mean([np.mean(sp) for sp in spans])) / N, 4)}
+
+    # ---- prefill, 40 layers
+    q = inputs.randn_cuda(3100, (1, H, N, D))
+    k = inputs.randn_cuda(3101, (1, H, N, D))
+    v = inputs.randn_cuda(3102, (1, H, N, D))
+    o = torch.empty_like(q)
+    ws = moa.Workspace(moa.MOA_OP_PREFILL, 1, H, N, D, spans[0])
+    pcaches = [moa.KVCache(1, H, D, "bf16", sp) for sp in spans]
+    flops = sum(prefill_flops(sp, N, D) for sp in spans)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+
+    def prefill_layers(record):
+        for layer in range(L):
+            if record:
+                ev[layer][0].record(stream)
+            moa.moa_prefill(q, k, v, o, 1, H, H, N, D, "bf16", spans[layer], scale, ws.ptr, ws.nbytes,
+                            pcaches[layer].handle, stream)
+            if record:
+                ev[layer][1].record(stream)
+
+    prefill_layers(False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler.for_current_device()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    prefill_layers(True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    p_clk = clocks.stop()
+    moa.moa_workspace_check(ws.ptr)
+    p_ms = e0.elapsed_time(e1)
+    p_kernel_ms = sum(a.elapsed_time(b) for a, b in ev)
+    tf = flops / (p_kernel_ms * 1e-3) / 1e12
+    out["prefill"] = {"layers": L, "ms": round(p_ms, 3), "ms_in_kernels": round(p_kernel_ms, 3),
+                      "in_window_flops": int(flops), "tflops": round(tf, 2),
+                      "roofline": {"bound": "tensor", "kernel": "prefill_bf16_sm100_kernel (moa_prefill + fill)",
+                                   "achieved": round(tf, 2), "peak": tf_peak, "unit": "TFLOP/s",
+                                   "frac": round(tf / tf_peak, 4), "peak_kind": peak_kind + " burst (bf16_tflops)",
+                                   "frac_of_sustained": round(tf / tf_sustained, 4)},
+                      "clocks": p_clk}
+    del q, k, v, o, pcaches
+    torch.cuda.empty_cache()
+
+    # ---- decode, 40 layers x V13_STEPS steps
+    caches, wss, dq, dk, dv, do = [], [], [], [], [], []
+    for layer in range(L):
+        c = moa.KVCache(B, H, D, "bf16", spans[layer])
+        data = c.data_bytes().view(torch.bfloat16)
+        for lo in range(0, data.numel(), 1 << 28):        # fill in slices: bounded temporaries
+            hi = min(data.numel(), lo + (1 << 28))
+            data[lo:hi].copy_(inputs.randn_cuda(3200 + layer * 64 + lo // (1 << 28), (hi - lo,)))
+        c.set_positions([N] * B)
+        caches.append(c)
+        wss.append(moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, D, spans[layer]))
+        dq.append(inputs.randn_cuda(3300 + layer, (B, H, D)))
+        dk.append(inputs.randn_cuda(3400 + layer, (B, H, 1, D)))
+        dv.append(inputs.randn_cuda(3500 + layer, (B, H, 1, D)))
+        do.append(torch.empty((B, H, D), dtype=torch.bfloat16, device="cuda"))
+    torch.cuda.synchronize()
+    layer_bytes = [B * sum(2 * S * D * 2 for S in sp) + 2 * B * H * D * 2 + 4 * B * H * D * 2 for sp in spans]
+    step_bytes = sum(layer_bytes)
+    kev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+           for _ in range(V13_STEPS)]
+
+    def dstep(i):
+        for layer in range(L):
+            if i is not None:
+                kev[i][layer][0].record(stream)
+            moa.moa_decode_append(caches[layer].handle, dq[layer], dk[layer], dv[layer], do[layer], H, spans[layer],
+                                  scale, wss[layer].ptr, wss[layer].nbytes, stream)
+            if i is not None:
+                kev[i][layer][1].record(stream)
+
+    for _ in range(3):
+        dstep(None)
+    torch.cuda.synchronize()
+    clocks = ClockSampler.for_current_device()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(V13_STEPS):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    d_clk = clocks.stop()
+    for c in caches:
+        c.positions()
+    d_ms = e0.elapsed_time(e1) / V13_STEPS
+    k_ms = sum(a.elapsed_time(b) for row in kev for a, b in row) / (V13_STEPS * L)
+    launch_gbs = (step_bytes / L) / (k_ms * 1e-3) / 1e9
+    out["decode"] = {"batch": B, "steps": V13_STEPS, "ms_per_step": round(d_ms, 4),
+                     "tokens_per_s": round(B / (d_ms * 1e-3), 2),
+                     "kv_gbs": round(step_bytes / (d_ms * 1e-3) / 1e9, 2), "bytes_per_step": int(step_bytes),
+                     "roofline": {"bound": "hbm", "kernel": "decode_kernel<bf16,128> (moa_decode_append)",
+                                  "achieved": round(launch_gbs, 2), "peak": hbm_peak, "unit": "GB/s",
+                                  "frac": round(launch_gbs / hbm_peak, 4), "peak_kind": peak_kind + " copy (hbm_gbs)",
+                                  "read_only_gbs": round(read_gbs, 1),
+                                  "frac_of_read_only": round(launch_gbs / read_gbs, 4)},
+                     "clocks": d_clk}
+    del caches, wss, dq, dk, dv, do
+    torch.cuda.empty_cache()
+    if with_cpu:
+        gf, n_rows = oracle_prefill_rate(spans[0], N, D, cpu_seconds / 2)
+        per_layer_s = oracle_decode_rate(spans[0], D, seqs=1)
+        out["cpu_baseline"] = {
+            "kind": "oracle", "cores": _oracle_threads(),
+            "prefill_gflops": round(gf, 4), "prefill_tflops": round(gf / 1e3, 7),
+            "prefill_sample": "%d query rows of layer 0 (every 97th row x every 4th head)" % n_rows,
+            "decode_tokens_per_s": round(1.0 / (per_layer_s * L), 5),
+            "decode_sample": "1 sequence x %d heads of layer 0 (fresh N(0,1) windows), time x %d layers" % (H, L)}
+    return out
+
+
+def llama3_gqa_prefill(stream, peaks, cpu_seconds, with_cpu, reps=20):
+    """Llama3-8B-shaped GQA prefill: 32 query heads on 8 KV heads, d=128, N=32768, B=1, spans per
+    query head at mean densities 12.5/25/50/100 % (100 % = dense causal), each KV group's cache
+    sized to the group's largest span and filled by the call.  Each density is timed back to back
+    (`reps` calls) in its own clock-sampled region."""
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    hbm_peak, tf_peak, tf_sustained, peak_kind = peaks
+    Hq, Hkv, N, D = L3_HQ, L3_HKV, L3_N, L3_D
+    G = Hq // Hkv
+    scale = 1.0 / math.sqrt(D)
+    q = inputs.randn_cuda(4100, (1, Hq, N, D))
+    k = inputs.randn_cuda(4101, (1, Hkv, N, D))
+    v = inputs.randn_cuda(4102, (1, Hkv, N, D))
+    o = torch.empty_like(q)
+    rows = []
+    all_spans = {}
+    for dens in L3_DENSITIES:
+        a, b = inputs.tables_7b(L3_SEED, Hq, N, BLOCK, dens, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, N, BLOCK)
+        all_spans[dens] = sp
+        caps = [max(sp[g * G:(g + 1) * G]) for g in range(Hkv)]
+        cache = moa.KVCache(1, Hkv, D, "bf16", caps)
+        ws = moa.Workspace(moa.MOA_OP_PREFILL, 1, Hq, N, D, sp)
+        flops = prefill_flops(sp, N, D)
+        ms, clk = back_to_back(stream, lambda: moa.moa_prefill(q, k, v, o, 1, Hq, Hkv, N, D, "bf16", sp, scale, ws.ptr,
+                                                               ws.nbytes, cache.handle, stream), reps)
+        moa.moa_workspace_check(ws.ptr)
+        cache.positions()
+        tf = flops / (ms * 1e-3) / 1e12
+        rows.append({"density": dens, "realised_density": round(float(np.mean(sp)) / N, 4),
+                     "capacities": caps, "ms": round(ms, 4), "in_window_flops": int(flops), "tflops": round(tf, 2),
+                     "frac": round(tf / tf_peak, 4), "frac_of_sustained": round(tf / tf_sustained, 4),
+                     "clocks": clk})
+        del cache, ws
+    out = {"workload": "llama3-8b-shaped GQA prefill: B=1, Hq=%d, Hkv=%d, d=%d, N=%d, spans per query head, "
+                       "group caches sized to the group's largest span and filled by the call" % (Hq, Hkv, D, N),
+           "kernel": "prefill_bf16_sm100_kernel (moa_prefill + fill)", "peak": tf_peak,
+           "peak_kind": peak_kind + " burst (bf16_tflops)", "reps": reps, "densities": rows}
+    if with_cpu:
+        gf, n_rows = oracle_prefill_rate(all_spans[0.25], N, D, cpu_seconds / 2, stride=389)
+        out["cpu_baseline"] = {
+            "kind": "oracle", "cores": _oracle_threads(), "gflops": round(gf, 4),
+            "sample": "%d query rows at density 0.25 (every 389th row x every 4th head); the other densities "
+                      "scaled by their in-window FLOPs" % n_rows,
+            "seconds_per_prompt": {str(r["density"]): round(r["in_window_flops"] / (gf * 1e9), 1) for r in rows}}
+    del q, k, v, o
+    torch.cuda.empty_cache()
+    return out
 
 
 def _ncu_traffic():
@@ -726,6 +1045,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--skip-extra", action="store_true",
+                    help="leave out the Vicuna-13B and Llama3-8B workloads (the 7B step and its entries only)")
     args = ap.parse_args()
     if args.profile_case:
         run_profile_case(args.profile_case)

@@ -36,6 +36,9 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* do
 moa_status cuda_fail(cudaError_t e, const char* where) {
   static const bool verbose = std::getenv("MOA_VERBOSE") != nullptr;
   if (verbose) std::fprintf(stderr, "libmoa: %s: %s\n", where, cudaGetErrorString(e));
+  // Clear the runtime's record of a non-sticky error here, so that a later
+  // launch check does not report it against an unrelated kernel.
+  (void)cudaGetLastError();
   return MOA_ERR_CUDA;
 }
 

@@ -37,12 +37,15 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 moa_status scratch_for_current_device(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOA_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return moa::cuda_fail(e, "static scratch: current device");
   if (dev < 0 || dev >= kMaxDevices) return MOA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return MOA_ERR_CUDA;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return moa::cuda_fail(e, "static scratch symbol");
+    if (p == nullptr) return moa::cuda_fail(cudaErrorInvalidSymbol, "static scratch symbol");
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -71,6 +74,7 @@ extern "C" moa_status moa_decode_static_ws(moa_kv_cache* c, const void* q, void*
   // The header and the per-(b, h) tickets must start at zero; the partials
   // are fully rewritten by every call.
   const size_t zero_bytes = 256 + (size_t)c->B * Hq * sizeof(uint32_t);
-  if (cudaMemsetAsync(scratch, 0, zero_bytes, s) != cudaSuccess) return MOA_ERR_CUDA;
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
+  if (e != cudaSuccess) return moa::cuda_fail(e, "static scratch memset");
   return moa::launch_decode(c, q, o, Hq, spans, scale, scratch, kStaticScratchBytes, s);
 }

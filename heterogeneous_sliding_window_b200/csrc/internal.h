@@ -44,7 +44,8 @@ int sm_count();
 cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* done);
 
 // MOA_ERR_CUDA with the CUDA error reported on stderr when the environment
-// variable MOA_VERBOSE is set (the status alone cannot carry the reason).
+// variable MOA_VERBOSE is set (the status alone cannot carry the reason);
+// clears the runtime's pending error.
 moa_status cuda_fail(cudaError_t e, const char* where);
 inline moa_status check_launch(const char* where) {
   const cudaError_t e = cudaGetLastError();

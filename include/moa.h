@@ -270,7 +270,8 @@ moa_status moa_decode_append(moa_kv_cache* cache, const void* q, const void* k, 
  * Decode without a caller workspace.  The paper has no counterpart: this is
  * a deployment convenience of this library.
  *
- * Same computation, arguments and errors as moa_decode, minus the workspace.
+ * Same computation, arguments and errors as moa_decode, minus the workspace
+ * (one more error below).
  * It is for callers that cannot allocate device memory -- e.g. an operator
  * plugin that its host framework gives only input and output pointers, a
  * runtime whose device memory is entirely owned by another allocator, or code
@@ -288,6 +289,8 @@ moa_status moa_decode_append(moa_kv_cache* cache, const void* q, const void* k, 
  *    device share the array, so calls whose work overlaps on the GPU (other
  *    streams, unordered threads) race and may return wrong outputs.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - Errors beyond moa_decode's: MOA_ERR_UNSUPPORTED when the current device
+ *    index is 64 or more (the per-device address table holds 64 devices).
  * ------------------------------------------------------------------------- */
 moa_status moa_decode_static_ws(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
                                 const int32_t* spans, float scale, void* stream);

@@ -126,6 +126,59 @@ def test_bf16_prefill_scores_growing_along_the_sequence():
     assert err <= BF16_TOL, err
 
 
+def test_bf16_prefill_scores_beyond_the_exponent_range():
+    """q x 16 and key norms growing to 12x along the sequence: scores reach several hundred
+    in log2 units, so 2^(s - m) overflows fp32 (ex2 gives inf above 128) unless the softmax
+    moves its reference first.  Element by element against the oracle, no NaN or inf."""
+    B, Hq, N, d = 1, 4, 900, 128
+    spans = [900, 300, 129, 640]
+    scale = 1.0 / math.sqrt(d)
+    q = (inputs.randn(41, (B, Hq, N, d), "f32") * 16.0).to(torch.bfloat16)
+    growth = torch.linspace(0.2, 12.0, N).view(1, 1, N, 1)
+    k = (inputs.randn(42, (B, Hq, N, d), "f32") * growth).to(torch.bfloat16)
+    v = inputs.randn(43, (B, Hq, N, d))
+    q64, k64, v64 = inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v)
+    s_max = max(float(np.max(q64[0, h] @ k64[0, h].T)) for h in range(Hq)) * scale * math.log2(math.e)
+    assert s_max > 128.0, s_max          # the case reaches past the exponent range
+    o = _bf16_prefill(q.to(DEV), k.to(DEV), v.to(DEV), spans, scale)
+    assert torch.isfinite(o.float()).all()
+    ref = oatt.prefill(q64, k64, v64, spans, scale)
+    err = np.max(np.abs(inputs.as_f64(o) - ref))
+    assert err <= BF16_TOL, err
+
+
+@pytest.mark.parametrize("Hkv", [4, 1], ids=["per_head", "group_mma"])
+def test_bf16_decode_scores_beyond_the_exponent_range(Hkv):
+    """Decode with q x 16 and cached keys up to 8x: scores far above 128 in log2 units, on the
+    per-head kernel and on the tensor-core group kernel."""
+    B, Hq, d, prefix = 2, 4, 128, 900
+    spans = [900, 513, 64, 700] if Hkv == 4 else [900, 880, 700, 600]
+    scale = 1.0 / math.sqrt(d)
+    caps = okv.group_capacities(spans, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+    ring = okv.RingCache(B, Hkv, d, caps)
+    growth = torch.linspace(1.0, 8.0, prefix).view(1, 1, prefix, 1)
+    k0 = (inputs.randn(44, (B, Hkv, prefix, d), "f32") * growth).to(torch.bfloat16)
+    v0 = inputs.randn(45, (B, Hkv, prefix, d))
+    cache.append(k0.to(DEV), v0.to(DEV))
+    ring.append(inputs.as_f64(k0), inputs.as_f64(v0))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, Hq, 0, d, spans)
+    for step in range(2):
+        qt = (inputs.randn(46 + step, (B, Hq, d), "f32") * 16.0).to(torch.bfloat16)
+        kt = (inputs.randn(48 + step, (B, Hkv, 1, d), "f32") * 8.0).to(torch.bfloat16)
+        vt = inputs.randn(50 + step, (B, Hkv, 1, d))
+        cache.append(kt.to(DEV), vt.to(DEV))
+        ring.append(inputs.as_f64(kt), inputs.as_f64(vt))
+        ot = _nan_like((B, Hq, d), torch.bfloat16)
+        moa.moa_decode(cache.handle, qt.to(DEV), ot, Hq, spans, scale, ws.ptr, ws.nbytes)
+        torch.cuda.synchronize()
+        assert torch.isfinite(ot.float()).all()
+        ref = okv.decode(ring, inputs.as_f64(qt), spans, scale)
+        err = np.max(np.abs(inputs.as_f64(ot) - ref))
+        assert err <= BF16_TOL, (step, err)
+    assert cache.positions() == ring.t
+
+
 def test_bf16_prefill_fill_cache_bytes():
     B, Hq, Hkv, N, d = 2, 4, 2, 600, 128
     spans = [64, 256, 600, 100]
@@ -288,6 +341,45 @@ def test_bf16_prefill_llama3_gqa_dense_sampled():
     ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale, rows=rows)
     got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
     assert np.max(np.abs(got - ref)) <= BF16_TOL
+
+
+def test_bf16_prefill_llama3_gqa_density_sweep_sampled():
+    """Hq=32 / Hkv=8, d=128, N=32768 at the sweep's 12.5, 25 and 50 % mean densities (per query
+    head spans, heterogeneous within each group), each KV group's cache sized to the group's
+    largest span and filled by the call, as the bench launches it; sampled rows, and the ring
+    bytes of sampled slots."""
+    B, Hq, Hkv, N, d = 1, 32, 8, 32768, 128
+    G = Hq // Hkv
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(4100, (B, Hq, N, d))
+    k = inputs.randn_cuda(4101, (B, Hkv, N, d))
+    v = inputs.randn_cuda(4102, (B, Hkv, N, d))
+    q64, k64, v64 = inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v)
+    rng = np.random.default_rng(5)
+    for dens in (0.125, 0.25, 0.5):
+        a, b = inputs.tables_7b(4000, Hq, N, 64, dens, orules.eval_spans)
+        spans = moa.moa_rules_eval(a, b, N, 64)
+        assert spans == orules.eval_spans(a, b, N, 64)
+        caps = okv.group_capacities(spans, Hkv)
+        cache = moa.KVCache(B, Hkv, d, "bf16", caps)
+        o = _bf16_prefill(q, k, v, spans, scale, fill=cache)
+        assert not torch.isnan(o).any()
+        rows = [(0, h, i) for h in (0, 9, 22, 31) for i in (0, 127, 128, 16383, N - 129, N - 1)]
+        rows += [(0, int(rng.integers(Hq)), int(rng.integers(N))) for _ in range(24)]
+        ref = oatt.prefill(q64, k64, v64, spans, scale, rows=rows)
+        got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
+        assert np.max(np.abs(got - ref)) <= BF16_TOL, dens
+        # the ring holds the last C_g positions of every group at slot p mod C_g
+        assert cache.positions() == [N]
+        data, goff = cache.layout()
+        blk = cache.data_bytes().view(torch.bfloat16)
+        for g in (0, Hkv - 1):
+            C = caps[g]
+            for p in (N - 1, N - C, N - 1 - int(rng.integers(C))):
+                base = goff[g] * 2 * d + (p % C) * d
+                assert torch.equal(blk[base:base + d].view(torch.int16), k[0, g, p].view(torch.int16))
+                assert torch.equal(blk[base + C * d:base + C * d + d].view(torch.int16), v[0, g, p].view(torch.int16))
+        del cache
 
 
 # ---------------------------------------------------------------------------
