@@ -21,8 +21,9 @@ where g = h // (Hq // Hkv) is the key/value head that query head h reads
 maximum leaves the result unchanged mathematically and keeps exp finite.
 
 Readings taken where the pages are silent: the window holds S_h keys including the
-query's own position (S_h = 1 attends to itself only); no sink or global
-tokens; spans are per query head.
+query's own position (S_h = 1 attends to itself only); spans are per query head.
+The plain path has no sink or global tokens; ``prefill_sink`` adds them (see
+there).
 
 Everything runs in numpy float64 on whatever values the caller passes
 (callers upcast the exact bf16 or fp32 values the GPU sees).
@@ -146,3 +147,86 @@ def in_window_flops(spans, N, d, B=1):
         pairs = S * N - S * (S - 1) // 2
         total += 4 * d * pairs
     return B * total
+
+
+# ---------------------------------------------------------------------------
+# Band plus global ("sink") tokens
+# ---------------------------------------------------------------------------
+# The codewithpapers page for arXiv 2406.14909 ("MoA: Mixture of Sparse
+# Attention for Automatic Large Language Model Compression") lists, from the
+# official repository, a pattern generator named gen_global_pattern beside
+# gen_band_pattern, and density counters named streamingllm_attention_density
+# and streamingllm_kv_cache_density; the project page's Table 4 compares with
+# StreamingLLM.  The pages give no formula.  Reading taken: a head with k_h
+# global tokens attends to its band and, in addition, to the first k_h
+# positions of the sequence (those that are causal), every key counted once:
+#
+#     keys(i) = { j : i - S_h < j <= i }  union  { j : 0 <= j < k_h, j <= i }
+#
+# k_h = 0 is the plain band; k_h >= N (or S_h >= N) is dense causal attention.
+
+
+def keys_sink(i, S, k):
+    """Sorted key positions of query row ``i`` under span ``S`` and ``k`` global tokens."""
+    if S < 1 or k < 0:
+        raise ValueError("span must be >= 1 and the global token count >= 0")
+    lo, hi = window(i, S)
+    band = set(range(lo, hi + 1))
+    glob = set(range(0, min(k, i + 1)))
+    return sorted(band | glob)
+
+
+def attend_keys(q_i, K, V, keys, scale):
+    """One output row: softmax over the listed key positions applied to their values."""
+    idx = np.asarray(keys, dtype=np.int64)
+    Ks = np.asarray(K, dtype=np.float64)[idx]
+    Vs = np.asarray(V, dtype=np.float64)[idx]
+    s = (Ks @ np.asarray(q_i, dtype=np.float64)) * scale
+    p = np.exp(s - s.max())
+    return (p / p.sum()) @ Vs
+
+
+def prefill_sink(q, k, v, spans, sinks, scale, rows=None):
+    """Windowed causal attention with global tokens over a whole prompt.
+
+    Same shapes and ``rows`` convention as ``prefill``; ``sinks`` holds k_h per
+    query head.  Row i of head h attends to ``keys_sink(i, S_h, k_h)``.
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    if len(spans) != Hq or len(sinks) != Hq:
+        raise ValueError("one span and one global token count per query head")
+    G = Hq // Hkv
+    if rows is None:
+        rows_list = [(b, h, i) for b in range(B) for h in range(Hq) for i in range(N)]
+    else:
+        rows_list = list(rows)
+    out = np.empty((len(rows_list), d), dtype=np.float64)
+    for n, (b, h, i) in enumerate(rows_list):
+        keys = keys_sink(i, int(spans[h]), int(sinks[h]))
+        out[n] = attend_keys(q[b, h, i], k[b, h // G], v[b, h // G], keys, scale)
+    if rows is None:
+        return out.reshape(B, Hq, N, d)
+    return out
+
+
+def in_window_flops_sink(spans, sinks, N, d, B=1):
+    """Algorithmic FLOPs of prefill with global tokens: 4 d per (row, key) pair.
+
+    Row i of head h touches min(i + 1, S_h) band keys and the global keys below
+    the band, max(0, min(k_h, i - S_h + 1)) of them.
+    """
+    total = 0
+    for S, kk in zip(spans, sinks):
+        S, kk = int(S), int(kk)
+        pairs = 0
+        for i in range(int(N)):
+            pairs += min(i + 1, S) + max(0, min(kk, i - S + 1))
+        total += 4 * d * pairs
+    return B * total
+

@@ -27,7 +27,10 @@ The device cache is one caller-owned buffer laid out as
 * header of ``align_up(16 + 8*B, 256)`` bytes: uint32 error word at byte 0,
   bytes 4..15 reserved, then int64 ``t[B]`` (tokens cached per sequence);
 * data: for b in 0..B-1, for g in 0..Hkv-1, the K block [C_g, d] followed by
-  the V block [C_g, d], row-major, elements of the cache dtype.
+  the V block [C_g, d], row-major, elements of the cache dtype;
+* for a cache that keeps global tokens (k_g of them for kv head g), after
+  that: for b, for g, Ksink [k_g, d] then Vsink [k_g, d], position p < k_g at
+  row p.
 
 :func:`data_image` rebuilds the data region byte for byte from this
 description so tests can compare the GPU buffer bit-exactly.
@@ -41,16 +44,23 @@ from .attention import attend_row
 class RingCache:
     """Python emulation of the per-(sequence, kv-head) ring buffers."""
 
-    def __init__(self, B, Hkv, d, capacities):
+    def __init__(self, B, Hkv, d, capacities, sinks=None):
         if len(capacities) != Hkv:
             raise ValueError("one capacity per kv head")
         if any(int(c) < 1 for c in capacities):
             raise ValueError("capacities must be >= 1")
+        sinks = [0] * Hkv if sinks is None else [int(x) for x in sinks]
+        if len(sinks) != Hkv or any(x < 0 for x in sinks):
+            raise ValueError("one global token count >= 0 per kv head")
         self.B, self.Hkv, self.d = int(B), int(Hkv), int(d)
         self.C = [int(c) for c in capacities]
         self.K = [[np.zeros((c, d), dtype=np.float64) for c in self.C] for _ in range(B)]
         self.V = [[np.zeros((c, d), dtype=np.float64) for c in self.C] for _ in range(B)]
         self.written = [[np.zeros(c, dtype=bool) for c in self.C] for _ in range(B)]
+        # global tokens: positions p < sinks[g] are also kept, for good, at sink slot p
+        self.sinks = sinks
+        self.Ks = [[np.zeros((x, d), dtype=np.float64) for x in sinks] for _ in range(B)]
+        self.Vs = [[np.zeros((x, d), dtype=np.float64) for x in sinks] for _ in range(B)]
         self.t = [0] * B
 
     @staticmethod
@@ -78,6 +88,9 @@ class RingCache:
                     self.K[b][g][s] = k[b, g, r]
                     self.V[b][g][s] = v[b, g, r]
                     self.written[b][g][s] = True
+                    if self.t[b] + r < self.sinks[g]:
+                        self.Ks[b][g][self.t[b] + r] = k[b, g, r]
+                        self.Vs[b][g][self.t[b] + r] = v[b, g, r]
             self.t[b] += n
 
     def window_positions(self, b, S):
@@ -96,6 +109,50 @@ class RingCache:
                 raise ValueError("position %d is not held by the ring" % p)
         idx = [self.slot(p, C) for p in positions]
         return self.K[b][g][idx], self.V[b][g][idx]
+
+
+    def gather_any(self, b, g, positions):
+        """K and V rows of the given positions, each read from the ring when the ring still
+        holds it, else from the global-token rows (positions below sinks[g])."""
+        C = self.C[g]
+        t = self.t[b]
+        Ks, Vs = [], []
+        for p in positions:
+            if t - C <= p < t:
+                Ks.append(self.K[b][g][self.slot(p, C)])
+                Vs.append(self.V[b][g][self.slot(p, C)])
+            elif 0 <= p < min(self.sinks[g], t):
+                Ks.append(self.Ks[b][g][p])
+                Vs.append(self.Vs[b][g][p])
+            else:
+                raise ValueError("position %d is held neither by the ring nor as a global token" % p)
+        return np.array(Ks), np.array(Vs)
+
+
+def decode_sink(cache, q, spans, sinks, scale):
+    """One decode step with global tokens: the query of position t = t_b - 1 of (b, h) attends
+    to keys_sink(t, S_h, k_h) of kv head g = h // (Hq // Hkv) (its band through the ring, the
+    first k_h positions through the global-token rows).  Needs S_h <= C_g and k_h <= sinks[g].
+    Returns float64 [B, Hq, d]."""
+    from .attention import keys_sink
+    q = np.asarray(q)
+    B, Hq, d = q.shape
+    if Hq % cache.Hkv != 0 or len(spans) != Hq or len(sinks) != Hq:
+        raise ValueError("shape mismatch")
+    G = Hq // cache.Hkv
+    out = np.empty((B, Hq, d), dtype=np.float64)
+    for b in range(B):
+        if cache.t[b] < 1:
+            raise ValueError("no tokens cached")
+        for h in range(Hq):
+            g = h // G
+            S, kk = int(spans[h]), int(sinks[h])
+            if S > cache.C[g] or kk > cache.sinks[g]:
+                raise ValueError("span or global token count exceeds the kv head's cache")
+            keys = keys_sink(cache.t[b] - 1, S, kk)
+            K, V = cache.gather_any(b, g, keys)
+            out[b, h] = attend_row(q[b, h], K, V, 0, len(keys) - 1, scale)
+    return out
 
 
 def decode(cache, q, spans, scale):
@@ -136,9 +193,10 @@ def header_bytes(B):
     return ((16 + 8 * int(B)) + 255) // 256 * 256
 
 
-def buffer_bytes(B, Hkv, d, capacities, elem_bytes):
-    """Total size of the device buffer for the documented layout."""
-    return header_bytes(B) + int(B) * sum(int(c) for c in capacities) * 2 * int(d) * int(elem_bytes)
+def buffer_bytes(B, Hkv, d, capacities, elem_bytes, sinks=None):
+    """Total size of the device buffer for the documented layout (global-token rows after the ring)."""
+    rows = sum(int(c) for c in capacities) + (sum(int(x) for x in sinks) if sinks else 0)
+    return header_bytes(B) + int(B) * rows * 2 * int(d) * int(elem_bytes)
 
 
 def _to_bits(x, dtype):
@@ -158,12 +216,18 @@ def _to_bits(x, dtype):
 
 
 def data_image(cache, dtype):
-    """Bytes of the data region: per b, per g, K[C_g, d] then V[C_g, d]."""
+    """Bytes of the data region: per b, per g, K[C_g, d] then V[C_g, d]; then, when the cache
+    keeps global tokens, per b, per g, Ksink[k_g, d] then Vsink[k_g, d] (slot p = position p)."""
     parts = []
     for b in range(cache.B):
         for g in range(cache.Hkv):
             parts.append(_to_bits(cache.K[b][g], dtype))
             parts.append(_to_bits(cache.V[b][g], dtype))
+    for b in range(cache.B):
+        for g in range(cache.Hkv):
+            if cache.sinks[g]:
+                parts.append(_to_bits(cache.Ks[b][g], dtype))
+                parts.append(_to_bits(cache.Vs[b][g], dtype))
     return b"".join(parts)
 
 

@@ -202,3 +202,66 @@ def test_flops_without_the_causal_triangle_is_caught(monkeypatch):
         return B * sum(4 * d * min(int(S), int(N)) * N for S in spans)   # dropped S(S-1)/2 term
     monkeypatch.setattr(attention, "in_window_flops", in_window_flops)
     assert _fails(ATT.test_in_window_flops_counts_mask_entries)
+
+
+# ---- band plus global tokens -------------------------------------------------
+SINK = _pins("test_oracle_sink")
+
+
+def _any_sink_brute_force_fails():
+    return any(_fails(SINK.test_sink_matches_brute_force_mask, c) for c in SINK.SINK_CASES)
+
+
+def _keys_mutant(glob_fn, join="union"):
+    def keys(i, S, k):
+        lo, hi = attention.window(i, S)
+        band = list(range(lo, hi + 1))
+        glob = list(glob_fn(i, k))
+        return sorted(set(band) | set(glob)) if join == "union" else sorted(band + glob)
+    return keys
+
+
+def test_sink_pins_pass_on_the_oracle_as_written():
+    assert not _any_sink_brute_force_fails()
+    for args in [(7, 3, 30), (16, 16, 40), (5, 9, 25)]:
+        assert not _fails(SINK.test_sink_decode_equals_last_prefill_row, *args)
+    assert not _fails(SINK.test_sink_image_layout_hand_computed)
+
+
+def test_global_range_one_too_wide_is_caught(monkeypatch):
+    monkeypatch.setattr(attention, "keys_sink", _keys_mutant(lambda i, k: range(0, min(k + 1, i + 1))))
+    assert _any_sink_brute_force_fails()
+
+
+def test_global_tokens_ignoring_causality_are_caught(monkeypatch):
+    monkeypatch.setattr(attention, "keys_sink", _keys_mutant(lambda i, k: range(0, k)))
+    assert _any_sink_brute_force_fails()
+
+
+def test_keys_in_band_and_global_counted_twice_is_caught(monkeypatch):
+    monkeypatch.setattr(attention, "keys_sink", _keys_mutant(lambda i, k: range(0, min(k, i + 1)), join="concat"))
+    assert _any_sink_brute_force_fails()
+
+
+def test_global_rows_read_through_the_ring_is_caught(monkeypatch):
+    def gather_ring_only(self, b, g, positions):
+        C = self.C[g]
+        idx = [p % C for p in positions]
+        return self.K[b][g][idx], self.V[b][g][idx]
+    monkeypatch.setattr(kvcache.RingCache, "gather_any", gather_ring_only)
+    assert any(_fails(SINK.test_sink_decode_equals_last_prefill_row, *a) for a in [(7, 3, 30), (5, 9, 25)])
+
+
+def test_global_rows_not_kept_at_append_is_caught(monkeypatch):
+    orig = kvcache.RingCache.append
+
+    def append_no_globals(self, k, v):
+        saved = self.sinks
+        self.sinks = [0] * self.Hkv
+        try:
+            orig(self, k, v)
+        finally:
+            self.sinks = saved
+    monkeypatch.setattr(kvcache.RingCache, "append", append_no_globals)
+    assert _fails(SINK.test_sink_image_layout_hand_computed)
+    assert any(_fails(SINK.test_sink_decode_equals_last_prefill_row, *a) for a in [(7, 3, 30), (5, 9, 25)])
