@@ -523,6 +523,7 @@ def run_ours(args):
     peaks = (hbm_peak, tf_peak, tf_sustained, peak_kind)
     v13 = vicuna13b(stream, peaks, read_gbs, args.cpu_seconds, rank == 0) if not args.skip_extra else None
     l3 = llama3_gqa_prefill(stream, peaks, args.cpu_seconds, rank == 0) if not args.skip_extra else None
+    glob = global_tokens(stream, peaks, read_gbs) if not args.skip_extra else None
 
     result = None
     if rank == 0:
@@ -567,6 +568,7 @@ def run_ours(args):
             "prefill_chunk": chunk,
             "vicuna13b": v13,
             "llama3_gqa_prefill": l3,
+            "global_tokens": glob,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clock_info,
             "cpu_baseline": {"value": round(cpu_tok, 4), "unit": "tokens/s", "cores": _oracle_threads(),
@@ -904,6 +906,78 @@ def llama3_gqa_prefill(stream, peaks, cpu_seconds, with_cpu, reps=20):
                       "scaled by their in-window FLOPs" % n_rows,
             "seconds_per_prompt": {str(r["density"]): round(r["in_window_flops"] / (gf * 1e9), 1) for r in rows}}
     del q, k, v, o
+    torch.cuda.empty_cache()
+    return out
+
+
+def sink_pairs(S, k, N):
+    """(row, key) pairs of one head with span S and k global tokens over N rows: the band's
+    sum_i min(i + 1, S), plus the global keys below the band, sum_i max(0, min(k, i - S + 1))."""
+    S, k = min(S, N), min(k, N)
+    band = S * N - S * (S - 1) // 2
+    n = N - S                              # rows whose band starts above position 0
+    extra = n * (n + 1) // 2 if n <= k else k * (k + 1) // 2 + k * (n - k)
+    return band + extra
+
+
+def global_tokens(stream, peaks, read_gbs, reps_prefill=100, reps_decode=300):
+    """Band plus global tokens on the Vicuna-7B shapes: the bench prompt (B=1, 32 heads, N=8192,
+    25 %) with per-head global tokens from {0, 4, 64, 128, 1024} and its cache fill, and one decode
+    layer (B=32, 32 heads, context 4096, 50 %) with the same draw, fused append + decode.  Each is
+    timed back to back in its own clock-sampled region."""
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    hbm_peak, tf_peak, tf_sustained, peak_kind = peaks
+    sinks = inputs.sink_counts(7, P_H)
+    # prefill
+    pa, pb = inputs.tables_7b(P_SEED, P_H, P_N, BLOCK, P_DENSITY, moa.moa_rules_eval)
+    sp = moa.moa_rules_eval(pa, pb, P_N, BLOCK)
+    q = inputs.randn_cuda(10, (P_B, P_H, P_N, P_D))
+    k = inputs.randn_cuda(11, (P_B, P_H, P_N, P_D))
+    v = inputs.randn_cuda(12, (P_B, P_H, P_N, P_D))
+    o = torch.empty_like(q)
+    ws = moa.Workspace(moa.MOA_OP_PREFILL, P_B, P_H, P_N, P_D, sp)
+    cache = moa.KVCache(P_B, P_H, P_D, "bf16", sp, sink_capacity=sinks)
+    scale = 1.0 / math.sqrt(P_D)
+    flops = 4 * P_D * sum(sink_pairs(S, kk, P_N) for S, kk in zip(sp, sinks)) * P_B
+    ms, clk = back_to_back(stream, lambda: moa.moa_prefill_sink(q, k, v, o, P_B, P_H, P_H, P_N, P_D, "bf16", sp,
+                                                                sinks, scale, ws.ptr, ws.nbytes, cache.handle,
+                                                                stream), reps_prefill)
+    moa.moa_workspace_check(ws.ptr)
+    cache.positions()
+    tf = flops / (ms * 1e-3) / 1e12
+    out = {"sinks": sinks,
+           "prefill": {"workload": "vicuna7b-shaped prompt B=1 H=32 d=128 N=8192 density 0.25 + global tokens, "
+                                   "cache fill", "ms": round(ms, 4), "in_window_flops": int(flops),
+                       "tflops": round(tf, 2), "frac": round(tf / tf_peak, 4),
+                       "peak_kind": peak_kind + " burst (bf16_tflops)", "clocks": clk}}
+    del q, k, v, o, ws, cache
+    # decode
+    a, b = inputs.tables_7b(D_SEED, D_H, D_N, BLOCK, D_DENSITY, moa.moa_rules_eval)
+    dsp = moa.moa_rules_eval(a, b, D_N, BLOCK)
+    c = moa.KVCache(D_B, D_H, D_D, "bf16", dsp, sink_capacity=sinks)
+    data = c.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(100, (data.numel(),)))
+    c.set_positions([D_N] * D_B)
+    nb = moa.moa_workspace_bytes_sink(moa.MOA_OP_DECODE, D_B, D_H, 0, D_D, dsp, sinks)
+    wbuf = torch.zeros(nb + 256, dtype=torch.uint8, device="cuda")
+    wptr = (wbuf.data_ptr() + 255) // 256 * 256
+    dq = inputs.randn_cuda(200, (D_B, D_H, D_D))
+    dk = inputs.randn_cuda(300, (D_B, D_H, 1, D_D))
+    dv = inputs.randn_cuda(400, (D_B, D_H, 1, D_D))
+    do = torch.empty_like(dq)
+    ms, clk = back_to_back(stream, lambda: moa.moa_decode_append_sink(c.handle, dq, dk, dv, do, D_H, dsp, sinks, scale,
+                                                                      wptr, nb, stream), reps_decode)
+    c.positions()
+    layer_bytes = D_B * sum(2 * (S + kk) * D_D * 2 for S, kk in zip(dsp, sinks)) + 6 * D_B * D_H * D_D * 2
+    gbs = layer_bytes / (ms * 1e-3) / 1e9
+    out["decode"] = {"workload": "vicuna7b-shaped decode layer B=32 H=32 d=128 ctx 4096 density 0.50 + global "
+                                 "tokens, fused append", "ms": round(ms, 4), "bytes_per_launch": int(layer_bytes),
+                     "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+                     "frac_of_read_only": round(gbs / read_gbs, 4),
+                     "tokens_per_s_one_layer": round(D_B / (ms * 1e-3), 1),
+                     "kernel": "decode_kernel<bf16,128> with global-token splits", "clocks": clk}
+    del c, wbuf
     torch.cuda.empty_cache()
     return out
 

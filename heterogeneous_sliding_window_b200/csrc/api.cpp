@@ -68,27 +68,44 @@ extern "C" moa_status moa_kv_header_bytes(int32_t B, size_t* bytes_out) {
   return MOA_OK;
 }
 
-extern "C" moa_status moa_kv_bytes(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
-                                   const int32_t* capacity, size_t* bytes_out) {
+extern "C" moa_status moa_kv_bytes_sink(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
+                                        const int32_t* capacity, const int32_t* sink_capacity,
+                                        size_t* bytes_out) {
   if (B < 1 || Hkv < 1 || Hkv > MOA_MAX_HEADS || !valid_d(d) || !valid_dtype(dtype) ||
       !capacity || !bytes_out)
     return MOA_ERR_INVALID_ARG;
-  int64_t sum = 0;
+  int64_t sum = 0, sum_sink = 0;
   for (int32_t g = 0; g < Hkv; ++g) {
     if (capacity[g] < 1) return MOA_ERR_INVALID_ARG;
     sum += capacity[g];
+    if (sink_capacity) {
+      if (sink_capacity[g] < 0) return MOA_ERR_INVALID_ARG;
+      sum_sink += sink_capacity[g];
+    }
   }
-  *bytes_out = header_bytes(B) + (size_t)B * (size_t)sum * 2 * (size_t)d * elem_bytes(dtype);
+  if (sum_sink > INT32_MAX) return MOA_ERR_INVALID_ARG;
+  *bytes_out = header_bytes(B) + (size_t)B * (size_t)(sum + sum_sink) * 2 * (size_t)d * elem_bytes(dtype);
   return MOA_OK;
+}
+
+extern "C" moa_status moa_kv_bytes(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
+                                   const int32_t* capacity, size_t* bytes_out) {
+  return moa_kv_bytes_sink(B, Hkv, d, dtype, capacity, nullptr, bytes_out);
 }
 
 extern "C" moa_status moa_kv_alloc(void* dev_buf, size_t bytes, int32_t B, int32_t Hkv, int32_t d,
                                    moa_dtype dtype, const int32_t* capacity, void* stream,
                                    moa_kv_cache** out) {
+  return moa_kv_alloc_sink(dev_buf, bytes, B, Hkv, d, dtype, capacity, nullptr, stream, out);
+}
+
+extern "C" moa_status moa_kv_alloc_sink(void* dev_buf, size_t bytes, int32_t B, int32_t Hkv, int32_t d,
+                                        moa_dtype dtype, const int32_t* capacity,
+                                        const int32_t* sink_capacity, void* stream, moa_kv_cache** out) {
   if (!out) return MOA_ERR_INVALID_ARG;
   *out = nullptr;
   size_t need = 0;
-  moa_status st = moa_kv_bytes(B, Hkv, d, dtype, capacity, &need);
+  moa_status st = moa_kv_bytes_sink(B, Hkv, d, dtype, capacity, sink_capacity, &need);
   if (st != MOA_OK) return st;
   if (!dev_buf || ((uintptr_t)dev_buf & 255u) != 0) return MOA_ERR_INVALID_ARG;
   if (bytes < need) return MOA_ERR_CAPACITY;
@@ -104,6 +121,11 @@ extern "C" moa_status moa_kv_alloc(void* dev_buf, size_t bytes, int32_t B, int32
   c->cap.assign(capacity, capacity + Hkv);
   c->goff.assign(Hkv + 1, 0);
   for (int32_t g = 0; g < Hkv; ++g) c->goff[g + 1] = c->goff[g] + capacity[g];
+  c->scap.assign(Hkv, 0);
+  if (sink_capacity) c->scap.assign(sink_capacity, sink_capacity + Hkv);
+  c->soff.assign(Hkv + 1, 0);
+  for (int32_t g = 0; g < Hkv; ++g) c->soff[g + 1] = c->soff[g] + c->scap[g];
+  c->sink_off = (size_t)B * (size_t)c->goff[Hkv] * 2 * (size_t)d * elem_bytes(dtype);
   if (cudaMemsetAsync(dev_buf, 0, need, (cudaStream_t)stream) != cudaSuccess) {
     delete c;
     return MOA_ERR_CUDA;
@@ -176,6 +198,18 @@ extern "C" moa_status moa_workspace_bytes(moa_op op, int32_t B, int32_t Hq, int6
   return MOA_ERR_INVALID_ARG;
 }
 
+extern "C" moa_status moa_workspace_bytes_sink(moa_op op, int32_t B, int32_t Hq, int64_t N, int32_t d,
+                                               const int32_t* spans, const int32_t* sinks, size_t* bytes_out) {
+  if (!sinks) return MOA_ERR_INVALID_ARG;
+  if (Hq >= 1 && Hq <= MOA_MAX_HEADS)
+    for (int32_t h = 0; h < Hq; ++h)
+      if (sinks[h] < 0) return MOA_ERR_INVALID_ARG;
+  const moa_status st = moa_workspace_bytes(op, B, Hq, N, d, spans, bytes_out);
+  if (st != MOA_OK || op != MOA_OP_DECODE) return st;
+  *bytes_out = decode_workspace_bytes(B, Hq, d, spans, sinks);
+  return MOA_OK;
+}
+
 extern "C" moa_status moa_workspace_init(void* ws, size_t bytes, void* stream) {
   if (!ws || bytes == 0) return MOA_ERR_INVALID_ARG;
   return cudaMemsetAsync(ws, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? MOA_OK : MOA_ERR_CUDA;
@@ -220,36 +254,70 @@ extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, con
   return MOA_OK;
 }
 
+static moa_status prefill_common(const void* q, const void* k, const void* v, void* o, int32_t B,
+                                 int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
+                                 const int32_t* spans, const int32_t* sinks, float scale, void* ws,
+                                 size_t ws_bytes, moa_kv_cache* fill, void* stream);
+
 extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, void* o, int32_t B,
                                   int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
                                   const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                   moa_kv_cache* fill, void* stream) {
+  return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, nullptr, scale, ws, ws_bytes, fill, stream);
+}
+
+extern "C" moa_status moa_prefill_sink(const void* q, const void* k, const void* v, void* o, int32_t B,
+                                       int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
+                                       const int32_t* spans, const int32_t* sinks, float scale, void* ws,
+                                       size_t ws_bytes, moa_kv_cache* fill, void* stream) {
+  if (!sinks) return MOA_ERR_INVALID_ARG;
+  return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, sinks, scale, ws, ws_bytes, fill, stream);
+}
+
+static moa_status prefill_common(const void* q, const void* k, const void* v, void* o, int32_t B,
+                                 int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
+                                 const int32_t* spans, const int32_t* sinks, float scale, void* ws,
+                                 size_t ws_bytes, moa_kv_cache* fill, void* stream) {
   if (!q || !k || !v || !o || !spans) return MOA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq > MOA_MAX_HEADS || Hkv > MOA_MAX_HEADS || Hq % Hkv != 0)
     return MOA_ERR_INVALID_ARG;
   if (N < 1 || N > INT32_MAX || !valid_d(d) || !valid_dtype(dtype)) return MOA_ERR_INVALID_ARG;
   if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
-  for (int32_t h = 0; h < Hq; ++h)
+  for (int32_t h = 0; h < Hq; ++h) {
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
+    if (sinks && sinks[h] < 0) return MOA_ERR_INVALID_ARG;
+  }
   const int32_t G = Hq / Hkv;
   if (fill) {
     if (fill->B != B || fill->Hkv != Hkv || fill->d != d || fill->dtype != dtype)
       return MOA_ERR_INVALID_ARG;
-    for (int32_t h = 0; h < Hq; ++h)
+    for (int32_t h = 0; h < Hq; ++h) {
       if (spans[h] > fill->cap[h / G]) return MOA_ERR_CAPACITY;
+      if (sinks && sinks[h] > fill->scap[h / G]) return MOA_ERR_CAPACITY;
+    }
   }
+  // global-token counts above N behave as N (and keep the kernels' arithmetic in range)
+  int32_t sk[MOA_MAX_HEADS];
+  bool any_sink = false;
+  if (sinks)
+    for (int32_t h = 0; h < Hq; ++h) {
+      sk[h] = (int32_t)std::min<int64_t>(sinks[h], N);
+      any_sink = any_sink || sk[h] > 0;
+    }
+  const int32_t* sinks_or_null = any_sink ? sk : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
   moa_status st;
   if (dtype == MOA_F32) {
     st = launch_prefill_f32((const float*)q, (const float*)k, (const float*)v, (float*)o, B, Hq, Hkv,
-                            (int32_t)N, d, spans, scale, s);
+                            (int32_t)N, d, spans, scale, s, sinks_or_null);
   } else {
     if (d != 128) return MOA_ERR_UNSUPPORTED;
     if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
     if (ws_bytes < prefill_workspace_bytes(B, Hq, N)) return MOA_ERR_WORKSPACE;
     // the kernel writes the cache itself
-    return launch_prefill_bf16(q, k, v, o, B, Hq, Hkv, (int32_t)N, spans, scale, ws, ws_bytes, s, fill);
+    return launch_prefill_bf16(q, k, v, o, B, Hq, Hkv, (int32_t)N, spans, scale, ws, ws_bytes, s, fill,
+                               sinks_or_null);
   }
   if (st != MOA_OK || !fill) return st;
   return launch_append(fill, k, v, (int32_t)N, s);
@@ -293,36 +361,58 @@ extern "C" moa_status moa_prefill_chunk(moa_kv_cache* c, const void* q, const vo
   return launch_prefill_chunk(c, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
 }
 
-extern "C" moa_status moa_decode_append(moa_kv_cache* c, const void* q, const void* k, const void* v,
-                                        void* o, int32_t Hq, const int32_t* spans, float scale, void* ws,
-                                        size_t ws_bytes, void* stream) {
-  if (!c || !q || !k || !v || !o || !spans) return MOA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+// Shared checks and dispatch of the decode entry points (k, v: the fused
+// append's new token, or both null; sinks: global tokens per query head, or
+// null).
+static moa_status decode_common(moa_kv_cache* c, const void* q, const void* k, const void* v, void* o,
+                                int32_t Hq, const int32_t* spans, const int32_t* sinks, float scale,
+                                void* ws, size_t ws_bytes, void* stream) {
+  if (!c || !q || !o || !spans) return MOA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
+  if ((k == nullptr) != (v == nullptr)) return MOA_ERR_INVALID_ARG;
+  if (k && (!aligned16(k) || !aligned16(v))) return MOA_ERR_INVALID_ARG;
   if (Hq < 1 || Hq > MOA_MAX_HEADS || Hq % c->Hkv != 0) return MOA_ERR_INVALID_ARG;
   if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
   const int32_t G = Hq / c->Hkv;
+  bool any_sink = false;
   for (int32_t h = 0; h < Hq; ++h) {
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
     if (spans[h] > c->cap[h / G]) return MOA_ERR_CAPACITY;
+    if (sinks) {
+      if (sinks[h] < 0) return MOA_ERR_INVALID_ARG;
+      if (sinks[h] > c->scap[h / G]) return MOA_ERR_CAPACITY;
+      any_sink = any_sink || sinks[h] > 0;
+    }
   }
+  const int32_t* sk = any_sink ? sinks : nullptr;
   if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
-  if (ws_bytes < decode_workspace_bytes(c->B, Hq, c->d, spans)) return MOA_ERR_WORKSPACE;
-  return launch_decode(c, q, o, Hq, spans, scale, ws, ws_bytes, (cudaStream_t)stream, k, v);
+  if (ws_bytes < decode_workspace_bytes(c->B, Hq, c->d, spans, sk)) return MOA_ERR_WORKSPACE;
+  return launch_decode(c, q, o, Hq, spans, scale, ws, ws_bytes, (cudaStream_t)stream, k, v, sk);
+}
+
+extern "C" moa_status moa_decode_append(moa_kv_cache* c, const void* q, const void* k, const void* v,
+                                        void* o, int32_t Hq, const int32_t* spans, float scale, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  if (!k || !v) return MOA_ERR_INVALID_ARG;
+  return decode_common(c, q, k, v, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream);
+}
+
+extern "C" moa_status moa_decode_append_sink(moa_kv_cache* c, const void* q, const void* k, const void* v,
+                                             void* o, int32_t Hq, const int32_t* spans, const int32_t* sinks,
+                                             float scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!k || !v || !sinks) return MOA_ERR_INVALID_ARG;
+  return decode_common(c, q, k, v, o, Hq, spans, sinks, scale, ws, ws_bytes, stream);
+}
+
+extern "C" moa_status moa_decode_sink(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
+                                      const int32_t* spans, const int32_t* sinks, float scale, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  if (!sinks) return MOA_ERR_INVALID_ARG;
+  return decode_common(c, q, nullptr, nullptr, o, Hq, spans, sinks, scale, ws, ws_bytes, stream);
 }
 
 extern "C" moa_status moa_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                                  const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                  void* stream) {
-  if (!c || !q || !o || !spans) return MOA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
-  if (Hq < 1 || Hq > MOA_MAX_HEADS || Hq % c->Hkv != 0) return MOA_ERR_INVALID_ARG;
-  if (!(scale == scale) || scale <= 0.f || scale > 1e30f) return MOA_ERR_INVALID_ARG;
-  const int32_t G = Hq / c->Hkv;
-  for (int32_t h = 0; h < Hq; ++h) {
-    if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
-    if (spans[h] > c->cap[h / G]) return MOA_ERR_CAPACITY;
-  }
-  if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
-  if (ws_bytes < decode_workspace_bytes(c->B, Hq, c->d, spans)) return MOA_ERR_WORKSPACE;
-  return launch_decode(c, q, o, Hq, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
+  return decode_common(c, q, nullptr, nullptr, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream);
 }

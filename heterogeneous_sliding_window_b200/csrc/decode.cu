@@ -59,6 +59,14 @@ struct DecodeParams {
   int32_t hslot_pre[MOA_MAX_HEADS + 1];   // group kernel: first partial slot of each query head
   int32_t cap[MOA_MAX_HEADS];
   int64_t goff[MOA_MAX_HEADS];
+  // Global tokens (per-head kernel only; sink_data == nullptr: none).  Head h
+  // has ceil(span/chunk) window splits, then ceil(sink[h]/chunk) splits over
+  // the global-token rows of its KV head (K_g = scap[g] rows at soff[g]).
+  char* sink_data;
+  int64_t sumK;
+  int32_t sink[MOA_MAX_HEADS];
+  int32_t scap[MOA_MAX_HEADS];
+  int64_t soff[MOA_MAX_HEADS];
 };
 
 template <typename T> struct Vec16;
@@ -134,16 +142,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int Seff = (int)(tb < (int64_t)p.span[h] ? tb : (int64_t)p.span[h]);
-  const int w0 = s * kChunk;
-  const int nrows = max(0, min(kChunk, Seff - w0));
+  const int nwin = (p.span[h] + kChunk - 1) / kChunk;  // window splits of head h
+  // Splits s >= nwin read the global tokens below the window: positions
+  // 0 .. min(k_h, tb - Seff) - 1, at rows of the same index.
+  const bool gsplit = s >= nwin;
+  const int w0 = (gsplit ? s - nwin : s) * kChunk;
+  const int nent = gsplit ? (int)min((int64_t)p.sink[h], tb - Seff) : Seff;
+  const int nrows = max(0, min(kChunk, nent - w0));
   const int64_t pos0 = tb - Seff + w0;                 // first window position of this split
-  const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
+  const int slot0 = gsplit ? w0 : nrows > 0 ? (int)(pos0 % C) : 0;
 
   T* Kb = reinterpret_cast<T*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
   T* Vb = Kb + (size_t)C * D;
+  if (gsplit) {
+    Kb = reinterpret_cast<T*>(p.sink_data) + (size_t)((int64_t)b * p.sumK + p.soff[g]) * 2 * D;
+    Vb = Kb + (size_t)p.scap[g] * D;
+  }
+  const int Cw = gsplit ? 0x7fffffff : C;              // global-token rows do not wrap
   // fused append: the newest window entry comes from the step's k, v, and the
-  // group's first head writes it to its slot
-  const int e_new = fused ? Seff - 1 : -1;
+  // group's first head writes it to its slot (and to its global-token row
+  // when its position is below K_g)
+  const int e_new = fused && !gsplit ? Seff - 1 : -1;
   const bool writer = fused && h == g * p.G;
   const T* kn = fused ? reinterpret_cast<const T*>(p.k_new) + ((size_t)b * (p.Hq / p.G) + g) * D : nullptr;
   const T* vn = fused ? reinterpret_cast<const T*>(p.v_new) + ((size_t)b * (p.Hq / p.G) + g) * D : nullptr;
@@ -171,13 +190,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       const int row = base + u * NG + grp;
       if (row < nrows) {
         int slot = slot0 + row;
-        if (slot >= C) slot -= C;
+        if (slot >= Cw) slot -= Cw;
         if (w0 + row == e_new) {
           kr[u] = __ldg(reinterpret_cast<const int4*>(kn + li * VE));
           vr[u] = __ldg(reinterpret_cast<const int4*>(vn + li * VE));
           if (writer) {
             *reinterpret_cast<int4*>(Kb + (size_t)slot * D + li * VE) = kr[u];
             *reinterpret_cast<int4*>(Vb + (size_t)slot * D + li * VE) = vr[u];
+            if (p.sink_data != nullptr && t0 < (int64_t)p.scap[g]) {
+              T* ks = reinterpret_cast<T*>(p.sink_data) + (size_t)((int64_t)b * p.sumK + p.soff[g]) * 2 * D +
+                      (size_t)t0 * D;
+              *reinterpret_cast<int4*>(ks + li * VE) = kr[u];
+              *reinterpret_cast<int4*>(ks + (size_t)p.scap[g] * D + li * VE) = vr[u];
+            }
           }
         } else {
           kr[u] = __ldcs(reinterpret_cast<const int4*>(Kb + (size_t)slot * D + li * VE));
@@ -925,15 +950,19 @@ struct DecodeLayout {
 // the group kernel sum_h ceil(C_g(h) / chunk); both are at most
 // Hq * ceil(max_h S_h / chunk), which sizes the workspace without knowing the
 // number of KV heads.
-DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* spans) {
+DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* spans, const int32_t* sinks) {
   DecodeLayout L;
-  int items = 0, max_s = 0;
+  int items = 0, max_s = 0, max_k = 0;
   for (int h = 0; h < Hq; ++h) {
     items += (spans[h] + kChunk - 1) / kChunk;
     max_s = max_s > spans[h] ? max_s : spans[h];
+    if (sinks) {
+      items += (sinks[h] + kChunk - 1) / kChunk;   // global-token splits
+      max_k = max_k > sinks[h] ? max_k : sinks[h];
+    }
   }
   L.items_per_b = items;
-  const size_t slots = (size_t)Hq * ((max_s + kChunk - 1) / kChunk);
+  const size_t slots = (size_t)Hq * ((max_s + kChunk - 1) / kChunk + (max_k + kChunk - 1) / kChunk);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   L.ctr_off = 256;
   L.bctr_off = L.ctr_off + up((size_t)B * Hq * 4);
@@ -945,14 +974,14 @@ DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* span
 
 }  // namespace
 
-size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans) {
-  return decode_layout(B, Hq, d, spans).total;
+size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans, const int32_t* sinks) {
+  return decode_layout(B, Hq, d, spans, sinks).total;
 }
 
 moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, const int32_t* spans,
                          float scale, void* ws, size_t ws_bytes, cudaStream_t s, const void* k_new,
-                         const void* v_new) {
-  const DecodeLayout L = decode_layout(c->B, Hq, c->d, spans);
+                         const void* v_new, const int32_t* sinks) {
+  const DecodeLayout L = decode_layout(c->B, Hq, c->d, spans, sinks);
   if (ws_bytes < L.total) return MOA_ERR_WORKSPACE;
   DecodeParams p;
   p.data = c->buf + c->header;
@@ -975,12 +1004,19 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   p.split_pre[0] = 0;
   for (int h = 0; h < Hq; ++h) {
     p.span[h] = spans[h];
-    p.split_pre[h + 1] = p.split_pre[h] + (spans[h] + kChunk - 1) / kChunk;
+    p.sink[h] = sinks ? sinks[h] : 0;
+    p.split_pre[h + 1] = p.split_pre[h] + (spans[h] + kChunk - 1) / kChunk + (p.sink[h] + kChunk - 1) / kChunk;
   }
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
     p.goff[g] = c->goff[g];
+    p.scap[g] = c->scap[g];
+    p.soff[g] = c->soff[g];
   }
+  // the cache's global-token rows are written by every fused append, also
+  // when this call attends to none of them
+  p.sink_data = sink_region(c);
+  p.sumK = c->soff[c->Hkv];
   // The group kernels read each cached row once for all G heads; the
   // per-head kernel reads overlapping windows once per head and L2 serves
   // most of the repeats.  bf16 with d = 128 and G = 2, 4 or 8 always takes
@@ -994,8 +1030,12 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   int64_t head_rows = 0, group_rows = 0;
   for (int h = 0; h < Hq; ++h) head_rows += spans[h];
   for (int g = 0; g < c->Hkv; ++g) group_rows += c->cap[g];
-  const bool mma_group = kGroupMma && c->dtype == MOA_BF16 && c->d == 128 && (G == 4 || G == 8 || (kGroupMma2 && G == 2));
-  if (mma_group || ((G == 4 || G == 8) && head_rows * 10 > group_rows * 22)) {
+  // Global tokens, and any cache that keeps global-token rows (the fused
+  // append writes them), take the per-head kernel.
+  const bool plain = p.sink_data == nullptr;
+  const bool mma_group = plain && kGroupMma && c->dtype == MOA_BF16 && c->d == 128 &&
+                         (G == 4 || G == 8 || (kGroupMma2 && G == 2));
+  if (mma_group || (plain && (G == 4 || G == 8) && head_rows * 10 > group_rows * 22)) {
     // group kernel: splits per KV group over its capacity, G partial slots each
     int items = 0;
     p.split_pre[0] = 0;

@@ -19,6 +19,12 @@ struct moa_kv_cache {
   size_t header = 0;             // bytes before the data region
   std::vector<int32_t> cap;      // C_g
   std::vector<int64_t> goff;     // prefix sums of C_g, size Hkv + 1
+  // global-token rows: K_g per key/value head (all 0: none), their prefix
+  // sums, and the region's byte offset from the start of the data region
+  std::vector<int32_t> scap;
+  std::vector<int64_t> soff;
+  size_t sink_off = 0;
+  bool has_sinks() const { return soff.empty() ? false : soff.back() > 0; }
 };
 
 namespace moa {
@@ -52,6 +58,12 @@ inline moa_status check_launch(const char* where) {
   return e == cudaSuccess ? MOA_OK : cuda_fail(e, where);
 }
 
+// Global-token region of a cache (nullptr when it keeps none) and, per key/value
+// head, its row count and row offset as the kernels take them.
+inline char* sink_region(const moa_kv_cache* c) {
+  return c->has_sinks() ? c->buf + c->header + c->sink_off : nullptr;
+}
+
 // kv.cu
 // Reads `bytes` (a multiple of 16) at 16-byte-aligned `buf` into a checksum
 // at `out` (one uint64 on the device).
@@ -59,16 +71,19 @@ moa_status launch_stream_read(const void* buf, size_t bytes, void* out, cudaStre
 moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t n_tok,
                          cudaStream_t s);
 
-// decode.cu
-size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans);
+// decode.cu.  sinks: global tokens per query head, or nullptr for none.
+size_t decode_workspace_bytes(int32_t B, int32_t Hq, int32_t d, const int32_t* spans,
+                              const int32_t* sinks = nullptr);
 moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                          const int32_t* spans, float scale, void* ws, size_t ws_bytes,
-                         cudaStream_t s, const void* k_new = nullptr, const void* v_new = nullptr);
+                         cudaStream_t s, const void* k_new = nullptr, const void* v_new = nullptr,
+                         const int32_t* sinks = nullptr);
 
 // prefill_simt.cu (fp32)
 moa_status launch_prefill_f32(const float* q, const float* k, const float* v, float* o,
                               int32_t B, int32_t Hq, int32_t Hkv, int32_t N, int32_t d,
-                              const int32_t* spans, float scale, cudaStream_t s);
+                              const int32_t* spans, float scale, cudaStream_t s,
+                              const int32_t* sinks = nullptr);
 
 // prefill_sm100.cu (bf16, tcgen05)
 constexpr int kTileM = 128;   // query rows per query tile (a work unit holds two)
@@ -81,8 +96,10 @@ struct PrefillSchedule {
   std::vector<int32_t> off;     // n_ctas + 1
   std::vector<int32_t> units;   // 4 int32 per unit
 };
+// sinks (nullable): global tokens per head; a query tile also visits the key
+// tiles below its band that hold them.
 PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
-                                 int32_t m0 = 0);
+                                 int32_t m0 = 0, const int32_t* sinks = nullptr);
 // Rows (CTA, unit, b, h, query tile, first key tile, last key tile), one per query tile.
 std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, const int32_t* spans,
                                            int32_t n_ctas);
@@ -93,7 +110,8 @@ size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N);
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o,
                                int32_t B, int32_t Hq, int32_t Hkv, int32_t N,
                                const int32_t* spans, float scale, void* ws, size_t ws_bytes,
-                               cudaStream_t s, moa_kv_cache* fill = nullptr);
+                               cudaStream_t s, moa_kv_cache* fill = nullptr,
+                               const int32_t* sinks = nullptr);
 
 // Self-test of the prefill kernel's bounded waits (prefill_sm100.cu): one CTA
 // on a 1 x 1 x 128 x 128 problem whose unit records are never published.

@@ -4,6 +4,8 @@
 // from a fixed-size KV cache sized per head.  Token position p of a sequence
 // is kept in slot p mod C_g of its key/value head g, so the buffer always
 // holds the last C_g tokens -- all that a head with span S_h <= C_g reads.
+// A cache that serves heads with global tokens also keeps positions p < K_g
+// for good, at row p of its global-token region.
 #include <algorithm>
 
 #include "internal.h"
@@ -24,6 +26,12 @@ struct AppendParams {
   int64_t sumC;
   int32_t cap[MOA_MAX_HEADS];
   int64_t goff[MOA_MAX_HEADS];
+  // global-token rows (sink == nullptr: none); blocks x >= ring_blocks copy them
+  char* sink;
+  int64_t sumK;
+  int32_t ring_blocks;
+  int32_t scap[MOA_MAX_HEADS];
+  int64_t soff[MOA_MAX_HEADS];
 };
 
 __global__ void __launch_bounds__(kAppendThreads) append_kernel(const __grid_constant__ AppendParams p) {
@@ -31,9 +39,29 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(const __grid_con
   const int b = blockIdx.z;
   const int C = p.cap[g];
   const int nrows = p.n_tok < C ? p.n_tok : C;   // only the last C rows survive
-  const int r0 = blockIdx.x * kAppendRows;
   const int64_t t0 = p.t[b];
-  if (r0 < nrows) {
+  if ((int)blockIdx.x >= p.ring_blocks) {
+    // global-token rows: token r at position t0 + r < K_g goes to row t0 + r
+    const int r0 = ((int)blockIdx.x - p.ring_blocks) * kAppendRows;
+    const int64_t lim = min((int64_t)p.n_tok, (int64_t)p.scap[g] - t0);
+    if (p.sink != nullptr && r0 < lim) {
+      const int rows = (int)min((int64_t)kAppendRows, lim - r0);
+      const int vpr = p.row_bytes / 16;
+      char* kdst = p.sink + (size_t)((int64_t)b * p.sumK + p.soff[g]) * 2 * p.row_bytes;
+      char* vdst = kdst + (size_t)p.scap[g] * p.row_bytes;
+      const size_t src_base = ((size_t)b * p.Hkv + g) * (size_t)p.n_tok;
+      for (int idx = threadIdx.x; idx < rows * vpr; idx += kAppendThreads) {
+        const int rr = idx / vpr;
+        const int vv = idx - rr * vpr;
+        const int r = r0 + rr;
+        const size_t src = (src_base + r) * p.row_bytes + (size_t)vv * 16;
+        const size_t dst = (size_t)(t0 + r) * p.row_bytes + (size_t)vv * 16;
+        *reinterpret_cast<int4*>(kdst + dst) = __ldg(reinterpret_cast<const int4*>(p.k + src));
+        *reinterpret_cast<int4*>(vdst + dst) = __ldg(reinterpret_cast<const int4*>(p.v + src));
+      }
+    }
+  } else if (blockIdx.x * kAppendRows < nrows) {
+    const int r0 = blockIdx.x * kAppendRows;
     const int rows = min(kAppendRows, nrows - r0);
     const int vpr = p.row_bytes / 16;
     const int first = p.n_tok - nrows;          // source row of the first survivor
@@ -153,14 +181,23 @@ moa_status launch_append(moa_kv_cache* c, const void* k, const void* v, int32_t 
   p.n_tok = n_tok;
   p.row_bytes = c->d * (int)elem_bytes(c->dtype);
   p.sumC = c->goff[c->Hkv];
-  int maxrows = 0;
+  int maxrows = 0, maxsink = 0;
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
     p.goff[g] = c->goff[g];
+    p.scap[g] = c->scap[g];
+    p.soff[g] = c->soff[g];
     const int r = n_tok < c->cap[g] ? n_tok : c->cap[g];
     if (r > maxrows) maxrows = r;
+    maxsink = std::max(maxsink, std::min(n_tok, c->scap[g]));
   }
-  dim3 grid((maxrows + kAppendRows - 1) / kAppendRows, c->Hkv, c->B);
+  p.sink = sink_region(c);
+  p.sumK = c->soff[c->Hkv];
+  p.ring_blocks = (maxrows + kAppendRows - 1) / kAppendRows;
+  // the global-token blocks cover the first min(n_tok, K_g) tokens; which of
+  // them land (positions below K_g) is decided on the device from t_b
+  const int sink_blocks = p.sink ? (maxsink + kAppendRows - 1) / kAppendRows : 0;
+  dim3 grid(p.ring_blocks + sink_blocks, c->Hkv, c->B);
   append_kernel<<<grid, kAppendThreads, 0, s>>>(p);
   return check_launch("append launch");
 }

@@ -134,6 +134,7 @@ struct PrefillParams {
   int32_t stall;                 // self-test of the bounded waits: the fetcher publishes nothing
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
+  int32_t sink[MOA_MAX_HEADS];   // global tokens per head (keys j < sink[h] are kept too), 0: none
   // Cache fill (fill_data == nullptr: none).  Row r of k_rows / v_rows
   // [B, Hkv, Nq, d] is position t_b + r of sequence b; the last min(Nq, C_g)
   // rows go to ring slot (t_b + r) mod C_g of KV head g, and the last CTA to
@@ -147,10 +148,15 @@ struct PrefillParams {
   int32_t B;
   int32_t fill_cap[MOA_MAX_HEADS];
   int64_t fill_goff[MOA_MAX_HEADS];
+  // Global-token rows of the cache (fill_sink == nullptr: none): positions
+  // below fill_scap[g] also go to row p of (b, g)'s block in this region.
+  char* fill_sink;
+  int64_t fill_sumK;             // sum of the global-token row counts
+  int32_t fill_scap[MOA_MAX_HEADS];
 };
-// The five tensor maps (128 bytes each) and the parameters share the 4 KB
-// kernel-parameter space.
-static_assert(sizeof(PrefillParams) + 5 * 128 <= 4096, "kernel parameters");
+// The five tensor maps (128 bytes each) and the parameters share the kernel
+// parameter space (32764 bytes on sm_70 and later since CUDA 12.1).
+static_assert(sizeof(PrefillParams) + 5 * 128 <= 32764, "kernel parameters");
 
 struct Ctx {
   uint32_t bar0;                       // address of barrier 0
@@ -214,17 +220,30 @@ __device__ __forceinline__ int first_key_tile(int t, int S) {
 }
 
 // The unit's two query tiles: X = 0 (A, tile m) and X = 1 (B, tile m + 1).
+// Query tile X visits the key tiles [0, min(ks, lo[X])) that hold global
+// tokens below its band, then its band [lo[X], m[X]].  The two tiles share
+// one stream of key tiles: the global prefix [0, P) with P = min(ks, lo[B]),
+// then [Lb, R] with Lb = max(lo[A], P).  Without global tokens (ks = 0) the
+// stream is lo[A] .. R.  Every stream tile up to m[A] belongs to tile A;
+// tile B skips the band tiles of A below lo[B].
 struct UnitInfo {
-  int S, zq, zk, kmin;
+  int S, k, zq, zk, kmin;
   int m[2], lo[2];
   bool hasB;
-  int L, R;                            // shared key-tile range
-  __device__ bool in(int X, int j) const { return (X == 0 || hasB) && j >= lo[X] && j <= m[X]; }
+  int ks;                              // key tiles t < ks hold global tokens
+  int P, Lb, R;                        // the shared key-tile stream (see above)
+  int start;                           // its first key tile
+  int first[2];                        // first key tile of each query tile
+  __device__ bool in(int X, int j) const {
+    return (X == 0 || hasB) && (j < ks || j >= lo[X]) && j <= m[X];
+  }
+  __device__ int next(int j) const { return j + 1 == P ? Lb : j + 1; }
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const int4 U, int kmin) {
   UnitInfo x;
   x.S = p.span[U.y];
+  x.k = p.sink[U.y];
   x.zq = U.x * p.Hq + U.y;
   x.zk = U.x * p.Hkv + U.y / p.G;
   x.kmin = kmin;
@@ -233,8 +252,13 @@ __device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const in
   x.m[1] = U.z + 1;
   x.hasB = (long long)x.m[1] * 128 < (long long)p.N;
   x.lo[1] = max(first_key_tile(x.m[1], x.S), kmin >> 7);
-  x.L = x.lo[0];
   x.R = x.hasB ? x.m[1] : x.m[0];
+  x.ks = (x.k + 127) >> 7;
+  x.P = min(x.ks, x.hasB ? x.lo[1] : x.lo[0]);
+  x.Lb = max(x.lo[0], x.P);
+  x.first[0] = x.ks > 0 ? 0 : x.lo[0];
+  x.first[1] = x.ks > 0 ? 0 : x.lo[1];
+  x.start = x.first[0];
   return x;
 }
 
@@ -256,24 +280,27 @@ constexpr float kSumHi = 32768.f;                    // 2^15
 constexpr float kSumLo = 1.f / 32768.f;              // 2^-15
 
 // 64 scores of half hh (columns 64hh .. 64hh+63) from tensor memory, masked.
-__device__ __forceinline__ void load_half(uint32_t tS, int hh, int hi_c, int lo_c, bool edge, float* s) {
+// Kept columns: lo_c < col <= hi_c (the band) and col < min(k_c, hi_c + 1)
+// (global tokens).  Returns whether the half keeps any column.
+__device__ __forceinline__ bool load_half(uint32_t tS, int hh, int hi_c, int lo_c, int k_c, bool edge,
+                                          float* s) {
   uint32_t sr[64];
   tmem_ld64(tS + 64u * (uint32_t)hh, sr);
 #pragma unroll
   for (int cc = 0; cc < 64; ++cc) s[cc] = __uint_as_float(sr[cc]);
-  if (edge) {
-    // Keep the columns lo_c < col <= hi_c: bits a..b of a 64-bit word built
-    // once per half, so each score costs one bit test and one select rather
-    // than two compares and a select (integer compares and selects issue at
-    // half the rate of the FMA pipe).
-    const int a = max(lo_c + 1 - 64 * hh, 0), b = min(hi_c - 64 * hh, 63);
-    const unsigned long long keep =
-        a > b ? 0ull : ((~0ull) >> (63 - max(b, 0))) & ((~0ull) << min(a, 63));
-    const uint32_t k0 = (uint32_t)keep, k1 = (uint32_t)(keep >> 32);
+  if (!edge) return true;
+  // Bits of a 64-bit word built once per half, so each score costs one bit
+  // test and one select rather than compares and a select (integer compares
+  // and selects issue at half the rate of the FMA pipe).
+  const int a = max(lo_c + 1 - 64 * hh, 0), b = min(hi_c - 64 * hh, 63);
+  unsigned long long keep = a > b ? 0ull : ((~0ull) >> (63 - max(b, 0))) & ((~0ull) << min(a, 63));
+  const int gb = min(min(k_c, hi_c + 1) - 1 - 64 * hh, 63);     // last global column of the half
+  if (gb >= 0) keep |= (~0ull) >> (63 - gb);
+  const uint32_t k0 = (uint32_t)keep, k1 = (uint32_t)(keep >> 32);
 #pragma unroll
-    for (int cc = 0; cc < 64; ++cc)
-      if (!(((cc < 32 ? k0 : k1) >> (cc & 31)) & 1u)) s[cc] = -INFINITY;
-  }
+  for (int cc = 0; cc < 64; ++cc)
+    if (!(((cc < 32 ? k0 : k1) >> (cc & 31)) & 1u)) s[cc] = -INFINITY;
+  return keep != 0ull;
 }
 
 __device__ __forceinline__ float max64(const float* s) {
@@ -339,22 +366,26 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
     // indexed so the unit record stays in registers
     const int m_x = X ? x.m[1] : x.m[0];
     const int lo_x = X ? x.lo[1] : x.lo[0];
+    const int s_x = min(x.ks, lo_x);                  // global tiles below the band: [0, s_x)
+    const int first_x = s_x > 0 ? 0 : lo_x;
     const int i_row = m_x * 128 + r;
     float m_run = -INFINITY, l_run = 0.f;            // m_run = -inf: no reference yet
-    for (int kt = lo_x; kt <= m_x; ++kt, ++tcount) {
+    for (int kt = first_x; kt <= m_x; kt = kt + 1 == s_x ? lo_x : kt + 1, ++tcount) {
       if (!c.wait_warp(B_SFULL0 + X, tcount & 1)) return;
       tc_fence_after();
       const int hi_c = i_row - kt * 128;             // keys c <= hi_c are causal
       const int lo_c = max(i_row - x.S, x.kmin - 1) - kt * 128;   // keys c > lo_c are inside the window
-      const bool edge = hi_c < 127 || lo_c >= 0;
+      const int k_c = x.k - kt * 128;                // keys c < k_c are global tokens
+      // every column kept: causal, and band and global tokens cover the tile
+      const bool full = hi_c >= 127 && (lo_c < 0 || k_c > lo_c || k_c >= 128);
+      const bool edge = !full;
       uint32_t w[64];                                // P of the tile, bf16 pairs
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float s[64];
-        load_half(tS, hh, hi_c, lo_c, edge, s);
+        const bool any_key = load_half(tS, hh, hi_c, lo_c, k_c, edge, s);
         const bool est = m_run != -INFINITY;
         float l_h = exp_half(s, sc, est ? -m_run : 0.f, w + 32 * hh);
-        const bool any_key = max(lo_c + 1, 64 * hh) <= min(hi_c, 64 * hh + 63);
         const bool bad = any_key && (!(l_h < kSumHi) || (!est && l_h < kSumLo));
         if (__any_sync(0xffffffffu, bad)) {
           // Rare: move the reference to this half's exact maximum.
@@ -365,9 +396,9 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
             m_run = mt;
             l_run *= alpha;
           }
-          if (kt > lo_x) {
-            // O holds every PV up to tile kt-1 (the S-ready commit of this
-            // tile covered them).
+          if (kt != first_x) {
+            // O holds every PV of the earlier tiles (the S-ready commit of
+            // this tile covered them).
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
               uint32_t rr[32];
@@ -485,11 +516,12 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
   if (U.x < 0) return;
   UnitInfo x = decode_unit(p, U, kmin);
   QSlots q = take_q(x, nq);
-  bool started_A = false;                            // S_A(L) of x already issued
+  bool started_A = false;                            // S_A(start) of x already issued
   while (true) {
     bool qrB = false;
-    // prologue: the S tiles of key tile L (tile A always starts at L; its S
-    // may have been issued during the previous unit's last step)
+    // prologue: the S tiles of the stream's first key tile (tile A always
+    // starts there; its S may have been issued during the previous unit's
+    // last step)
     if (!c.wait(B_KFULL0 + kst, kph)) return;
     {
       const uint32_t dk = desc_qk_lo(sK0 + kst * kTileBytes);
@@ -498,9 +530,9 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
         tc_fence_after();
         mma_qk(tSA, desc_qk_lo(sQ0 + q.sA * kTileBytes), dk, hi);
         mma_commit(c.bar(B_SFULL0));
-        if (x.L == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
+        if (x.start == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
       }
-      if (x.in(1, x.L)) {
+      if (x.in(1, x.start)) {
         if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
         qrB = true;
         tc_fence_after();
@@ -515,16 +547,17 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     int4 Uy = make_int4(0, 0, 0, 0);
     int ykmin = 0;
     uint32_t ysA = 0, ypA = 0;
-    for (int j = x.L; j <= x.R; ++j) {
+    for (int j = x.start;; ) {
       const bool more = j < x.R;
+      const int jn = x.next(j);                      // the stream's next key tile, when more
       if (!c.wait(B_VFULL0 + vst, vph)) return;
       const uint32_t dv = desc_v_lo(sV0 + vst * kTileBytes);
-      const uint32_t dk = desc_qk_lo(sK0 + kst * kTileBytes);   // K(j+1) when more
+      const uint32_t dk = desc_qk_lo(sK0 + kst * kTileBytes);   // K(jn) when more
       if (more && !c.wait(B_KFULL0 + kst, kph)) return;
-      // stream A: O_A += P_A(j) V(j), then S_A(j+1)
+      // stream A: O_A += P_A(j) V(j), then S_A(jn)
       if (j <= x.m[0]) {
         if (!c.wait(B_PFULL0, tpA & 1)) return;
-        const bool first = j == x.lo[0];
+        const bool first = j == x.first[0];
         if (first && !c.wait(B_OEMPTY0, (ucA & 1) ^ 1)) return;
         tc_fence_after();
         mma_pv(tOA, tSA, dv, hi, first);
@@ -533,9 +566,9 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
           mma_commit(c.bar(B_OFULL0));
           ++ucA;
         } else {
-          mma_qk(tSA, desc_qk_lo(sQ0 + q.sA * kTileBytes), dk, hi);   // j + 1 <= m_A, so more
+          mma_qk(tSA, desc_qk_lo(sQ0 + q.sA * kTileBytes), dk, hi);   // jn <= m_A, so more
           mma_commit(c.bar(B_SFULL0));               // also covers PV_A(j)
-          if (j + 1 == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
+          if (jn == x.m[0]) mma_commit(c.bar(B_QEMPTY0 + q.sA));
         }
       } else if (!more) {
         // Last step, tile B only: S_A of the next unit's first key tile (the
@@ -554,15 +587,16 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
           tc_fence_after();
           mma_qk(tSA, desc_qk_lo(sQ0 + ysA * kTileBytes), desc_qk_lo(sK0 + kst * kTileBytes), hi);
           mma_commit(c.bar(B_SFULL0));
-          if (max(Uy.w, ykmin >> 7) == Uy.z) mma_commit(c.bar(B_QEMPTY0 + ysA));
+          const UnitInfo y = decode_unit(p, Uy, ykmin);
+          if (y.start == y.m[0]) mma_commit(c.bar(B_QEMPTY0 + ysA));
           have_next = true;
         }
       }
-      // stream B: O_B += P_B(j) V(j), then S_B(j+1)
+      // stream B: O_B += P_B(j) V(j), then S_B(jn)
       if (x.hasB) {
-        if (j >= x.lo[1]) {
+        if (x.in(1, j)) {
           if (!c.wait(B_PFULL0 + 1, tpB & 1)) return;
-          const bool first = j == x.lo[1];
+          const bool first = j == x.first[1];
           if (first && !c.wait(B_OEMPTY0 + 1, (ucB & 1) ^ 1)) return;
           tc_fence_after();
           mma_pv(tOB, tSB, dv, hi, first);
@@ -572,7 +606,7 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
             ++ucB;
           }
         }
-        if (more && j + 1 >= x.lo[1]) {
+        if (more && x.in(1, jn)) {
           if (!qrB) {
             if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
             qrB = true;
@@ -580,15 +614,15 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
           }
           mma_qk(tSB, desc_qk_lo(sQ0 + q.sB * kTileBytes), dk, hi);
           mma_commit(c.bar(B_SFULL0 + 1));
-          if (j + 1 == x.m[1]) mma_commit(c.bar(B_QEMPTY0 + q.sB));
+          if (jn == x.m[1]) mma_commit(c.bar(B_QEMPTY0 + q.sB));
         }
       }
       mma_commit(c.bar(B_VEMPTY0 + vst));
       if (++vst == kVStages) { vst = 0; vph ^= 1u; }
-      if (more) {
-        mma_commit(c.bar(B_KEMPTY0 + kst));
-        if (++kst == kKStages) { kst = 0; kph ^= 1u; }
-      }
+      if (!more) break;
+      mma_commit(c.bar(B_KEMPTY0 + kst));
+      if (++kst == kKStages) { kst = 0; kph ^= 1u; }
+      j = jn;
     }
     if (ended) return;
     if (have_next) {
@@ -655,17 +689,18 @@ __device__ __forceinline__ void producer_role(const PrefillParams& p, const Ctx&
     if (!c.next_unit(i, 0, false, &U, &kmin)) return;
     if (U.x < 0) return;
     const UnitInfo x = decode_unit(p, U, kmin);
-    // Loads in the MMA's order of use: Q_A, K(L), then per key tile j:
-    // V(j), K(j+1); Q_B right before the first K tile that tile B uses.
+    // Loads in the MMA's order of use: Q_A, K(start), then per key tile j
+    // of the stream: V(j), K(next); Q_B right before the first K tile that
+    // tile B uses.
     if (!load_q(x.m[0], x.zq)) return;
-    if (!load_k(x.L, x.zk)) return;
-    if (x.hasB && x.lo[1] == x.L && !load_q(x.m[1], x.zq)) return;
-    for (int j = x.L; j <= x.R; ++j) {
+    if (!load_k(x.start, x.zk)) return;
+    if (x.hasB && x.first[1] == x.start && !load_q(x.m[1], x.zq)) return;
+    for (int j = x.start;; j = x.next(j)) {
       if (!load_v(j, x.zk)) return;
-      if (j < x.R) {
-        if (x.hasB && x.lo[1] == j + 1 && !load_q(x.m[1], x.zq)) return;
-        if (!load_k(j + 1, x.zk)) return;
-      }
+      if (j >= x.R) break;
+      const int jn = x.next(j);
+      if (x.hasB && x.first[1] == jn && !load_q(x.m[1], x.zq)) return;
+      if (!load_k(jn, x.zk)) return;
     }
   }
 }
@@ -716,6 +751,23 @@ __device__ __forceinline__ void fill_role(const PrefillParams& p, int lane) {
     const int g = U.y / p.G;
     const int C = p.fill_cap[g];
     const int q0 = U.z * 128 - p.q_off;              // the unit's first query row
+    if (p.fill_sink != nullptr && p.fill_scap[g] > 0) {
+      // global-token rows: positions t_b + r below K_g, at row t_b + r of (b, g)'s block
+      const int64_t tb = p.fill_t[U.x];
+      const int Kg = p.fill_scap[g];
+      const int g_end = (int)min((int64_t)min(q0 + 256, p.Nq), (int64_t)Kg - tb);
+      int64_t soff = 0;
+      for (int gg = 0; gg < g; ++gg) soff += p.fill_scap[gg];
+      char* ks = p.fill_sink + (size_t)((int64_t)U.x * p.fill_sumK + soff) * 2 * kRowBytes;
+      char* vs = ks + (size_t)Kg * kRowBytes;
+      const size_t src0 = ((size_t)U.x * p.Hkv + g) * (size_t)p.Nq;
+      for (int r = q0 + half; r < g_end; r += 2) {
+        const size_t src = (src0 + r) * kRowBytes + col;
+        const size_t dst = (size_t)(tb + r) * kRowBytes + col;
+        *reinterpret_cast<int4*>(ks + dst) = __ldg(reinterpret_cast<const int4*>(p.k_rows + src));
+        *reinterpret_cast<int4*>(vs + dst) = __ldg(reinterpret_cast<const int4*>(p.v_rows + src));
+      }
+    }
     const int r_first = max(q0, p.Nq - C);           // rows below Nq - C are overwritten later
     const int r_end = min(q0 + 256, p.Nq);
     if (r_first >= r_end) continue;
@@ -878,7 +930,7 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 // time rule (each unit to the list with the least work so far); a unit's work
 // is its (query tile, key tile) pairs plus a fixed per-unit overhead.
 PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
-                                 int32_t m0) {
+                                 int32_t m0, const int32_t* sinks) {
   const int64_t M = (N + kTileM - 1) / kTileM;      // key tiles; query tiles are m0 .. M-1
   const int64_t per_head = std::max<int64_t>(0, (M - m0 + 1) / 2);
   const int64_t n_units = (int64_t)B * Hq * per_head;
@@ -889,8 +941,13 @@ PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t
     for (int64_t k = 0; k < per_head; ++k) {
       const int64_t m = m0 + 2 * k;
       const int64_t l = first_tile_host(m, spans[h]);
-      int64_t c = m - l + 1 + kUnitOverheadTiles;
-      if (m + 1 < M) c += m + 1 - first_tile_host(m + 1, spans[h]) + 1;
+      // key tiles below the band that hold global tokens
+      const int64_t ks = sinks ? ((int64_t)sinks[h] + kTileN - 1) / kTileN : 0;
+      int64_t c = m - l + 1 + std::min(ks, l) + kUnitOverheadTiles;
+      if (m + 1 < M) {
+        const int64_t lb = first_tile_host(m + 1, spans[h]);
+        c += m + 1 - lb + 1 + std::min(ks, lb);
+      }
       for (int32_t b = 0; b < B; ++b) {
         const size_t u = (size_t)(((int64_t)b * Hq + h) * per_head + k);
         lo[u] = (int32_t)l;
@@ -988,18 +1045,20 @@ struct UnitBlob {
 
 struct BlobKey {
   int32_t B, Hq, N, grid, m0;
-  std::vector<int32_t> spans;
+  std::vector<int32_t> spans, sinks;
   bool operator==(const BlobKey& o) const {
-    return B == o.B && Hq == o.Hq && N == o.N && grid == o.grid && m0 == o.m0 && spans == o.spans;
+    return B == o.B && Hq == o.Hq && N == o.N && grid == o.grid && m0 == o.m0 && spans == o.spans &&
+           sinks == o.sinks;
   }
 };
 
 std::shared_ptr<const UnitBlob> unit_blob(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t grid,
-                                          int32_t m0) {
+                                          int32_t m0, const int32_t* sinks) {
   constexpr size_t kKept = 8;
   static std::mutex mu;
   static std::vector<std::pair<BlobKey, std::shared_ptr<const UnitBlob>>> kept;   // most recent first
-  BlobKey key{B, Hq, N, grid, m0, std::vector<int32_t>(spans, spans + Hq)};
+  BlobKey key{B, Hq, N, grid, m0, std::vector<int32_t>(spans, spans + Hq),
+              sinks ? std::vector<int32_t>(sinks, sinks + Hq) : std::vector<int32_t>()};
   {
     std::lock_guard<std::mutex> lock(mu);
     for (size_t i = 0; i < kept.size(); ++i)
@@ -1008,7 +1067,7 @@ std::shared_ptr<const UnitBlob> unit_blob(int32_t B, int32_t Hq, int32_t N, cons
         return kept[0].second;
       }
   }
-  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, grid, m0);
+  const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, grid, m0, sinks);
   auto blob = std::make_shared<UnitBlob>();
   blob->n_ctas = sch.n_ctas;
   blob->words.assign(kUnitsOffset / 4 + sch.units.size(), 0);
@@ -1030,7 +1089,8 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
                                     int32_t q_off, const int64_t* t, const int32_t* spans, float scale,
                                     void* ws, size_t ws_bytes, cudaStream_t s, moa_kv_cache* fill = nullptr,
                                     bool stall = false,
-                                    const std::function<moa_status()>& before = nullptr) {
+                                    const std::function<moa_status()>& before = nullptr,
+                                    const int32_t* sinks = nullptr) {
   if (ws_bytes < prefill_workspace_bytes(B, Hq, Nq)) return MOA_ERR_WORKSPACE;
   if ((int64_t)B * Hq > INT32_MAX || (int64_t)B * Hkv > INT32_MAX) return MOA_ERR_UNSUPPORTED;
   const int32_t Nk = q_off + Nq;
@@ -1052,7 +1112,7 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   const int64_t Mq = (Nq + kTileM - 1) / kTileM;
   const int64_t n_units = (int64_t)B * Hq * ((Mq + 1) / 2);
   const int32_t grid = (int32_t)std::min<int64_t>({n_units, (int64_t)sm_count(), (int64_t)kPrefillMaxCtas});
-  const std::shared_ptr<const UnitBlob> sch = unit_blob(B, Hq, Nk, spans, grid, m0);
+  const std::shared_ptr<const UnitBlob> sch = unit_blob(B, Hq, Nk, spans, grid, m0, sinks);
   const std::vector<int32_t>& blob = sch->words;
 
   PrefillParams p;
@@ -1069,7 +1129,10 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.scale_log2 = scale * 1.4426950408889634f;
-  for (int h = 0; h < Hq; ++h) p.span[h] = spans[h];
+  for (int h = 0; h < Hq; ++h) {
+    p.span[h] = spans[h];
+    p.sink[h] = sinks ? sinks[h] : 0;
+  }
   p.B = B;
   p.fill_data = nullptr;
   p.fill_ctr = nullptr;
@@ -1077,6 +1140,8 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.k_rows = static_cast<const char*>(k);
   p.v_rows = static_cast<const char*>(v);
   p.fill_sumC = 0;
+  p.fill_sink = nullptr;
+  p.fill_sumK = 0;
   if (fill != nullptr) {
     if (fill->B != B || fill->Hkv != Hkv || fill->d != kD || fill->dtype != MOA_BF16) return MOA_ERR_INVALID_ARG;
     p.fill_data = fill->buf + fill->header;
@@ -1086,7 +1151,10 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
     for (int g = 0; g < Hkv; ++g) {
       p.fill_cap[g] = fill->cap[g];
       p.fill_goff[g] = fill->goff[g];
+      p.fill_scap[g] = fill->scap[g];
     }
+    p.fill_sink = sink_region(fill);
+    p.fill_sumK = fill->soff[Hkv];
   }
 
   static unsigned long long attr_done = 0;
@@ -1130,9 +1198,10 @@ ChunkLayout chunk_layout(int32_t B, int32_t Hq, int32_t Hkv, int32_t n, const in
 
 moa_status launch_prefill_bf16(const void* q, const void* k, const void* v, void* o, int32_t B,
                                int32_t Hq, int32_t Hkv, int32_t N, const int32_t* spans, float scale,
-                               void* ws, size_t ws_bytes, cudaStream_t s, moa_kv_cache* fill) {
+                               void* ws, size_t ws_bytes, cudaStream_t s, moa_kv_cache* fill,
+                               const int32_t* sinks) {
   return launch_prefill_bf16_rows(q, k, v, nullptr, nullptr, o, B, Hq, Hkv, N, 0, nullptr, spans, scale, ws,
-                                  ws_bytes, s, fill);
+                                  ws_bytes, s, fill, false, nullptr, sinks);
 }
 
 moa_status launch_prefill_stall_test(const void* q, const void* k, const void* v, void* o, void* ws,

@@ -119,3 +119,15 @@ def tables_13b_mix(seed, n_heads, N, block, density, rules_fn):
 def tiny_tables():
     """Tiny fp32 case: 4 heads with spans {32, 64, 128, 256} (beta = 0, block 32)."""
     return np.array([32.0, 64.0, 128.0, 256.0]), np.zeros(4)
+
+
+# Global-token counts per head for the band-plus-global-token workloads: a
+# seeded draw from a small set (a few StreamingLLM-style sink tokens up to a
+# few tiles of them).
+SINK_SET = (0, 4, 64, 128, 1024)
+
+
+def sink_counts(seed, n_heads, choices=SINK_SET):
+    """Per-head global token counts drawn uniformly from ``choices``."""
+    rng = np.random.default_rng(seed)
+    return [int(x) for x in rng.choice(np.asarray(choices, dtype=np.int64), size=n_heads)]

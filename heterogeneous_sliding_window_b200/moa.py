@@ -25,7 +25,8 @@ EXPORTS = (
     "moa_kv_free", "moa_kv_append", "moa_kv_positions", "moa_kv_set_positions", "moa_kv_layout",
     "moa_workspace_bytes", "moa_workspace_init", "moa_workspace_check", "moa_prefill",
     "moa_prefill_schedule", "moa_decode", "moa_decode_append", "moa_decode_static_ws", "moa_stream_read", "moa_chunk_workspace_bytes",
-    "moa_prefill_chunk", "moa_prefill_stall_test",
+    "moa_prefill_chunk", "moa_prefill_stall_test", "moa_kv_bytes_sink", "moa_kv_alloc_sink", "moa_prefill_sink",
+    "moa_workspace_bytes_sink", "moa_decode_sink", "moa_decode_append_sink",
 )
 
 
@@ -72,6 +73,13 @@ def load():
         "moa_prefill_stall_test": (ctypes.c_int, [vp, vp, vp, vp, vp, sz, vp]),
         "moa_chunk_workspace_bytes": (ctypes.c_int, [vp, i32, i32, P(i32), P(sz)]),
         "moa_prefill_chunk": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, i32, P(i32), f32, vp, sz, vp]),
+        "moa_kv_bytes_sink": (ctypes.c_int, [i32, i32, i32, ctypes.c_int, P(i32), P(i32), P(sz)]),
+        "moa_kv_alloc_sink": (ctypes.c_int, [vp, sz, i32, i32, i32, ctypes.c_int, P(i32), P(i32), vp, P(vp)]),
+        "moa_prefill_sink": (ctypes.c_int, [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_int, P(i32), P(i32),
+                                            f32, vp, sz, vp, vp]),
+        "moa_workspace_bytes_sink": (ctypes.c_int, [ctypes.c_int, i32, i32, i64, i32, P(i32), P(i32), P(sz)]),
+        "moa_decode_sink": (ctypes.c_int, [vp, vp, vp, i32, P(i32), P(i32), f32, vp, sz, vp]),
+        "moa_decode_append_sink": (ctypes.c_int, [vp, vp, vp, vp, vp, i32, P(i32), P(i32), f32, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -266,19 +274,76 @@ def moa_stream_read(buf, nbytes, out, stream=None):
     _check(load().moa_stream_read(_ptr(buf), int(nbytes), _ptr(out), _stream(stream)), "moa_stream_read")
 
 
+# ---- band plus global tokens ------------------------------------------------
+def moa_kv_bytes_sink(B, Hkv, d, dtype, capacity, sink_capacity):
+    cap, cp = _i32(capacity)
+    sk, skp = _i32(sink_capacity)
+    out = ctypes.c_size_t()
+    _check(load().moa_kv_bytes_sink(B, Hkv, d, _dtype(dtype), cp, skp, ctypes.byref(out)), "moa_kv_bytes_sink")
+    return out.value
+
+
+def moa_kv_alloc_sink(buf, nbytes, B, Hkv, d, dtype, capacity, sink_capacity, stream=None):
+    cap, cp = _i32(capacity)
+    sk, skp = _i32(sink_capacity)
+    h = ctypes.c_void_p()
+    _check(load().moa_kv_alloc_sink(_ptr(buf), nbytes, B, Hkv, d, _dtype(dtype), cp, skp, _stream(stream),
+                                    ctypes.byref(h)), "moa_kv_alloc_sink")
+    return h
+
+
+def moa_prefill_sink(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, sinks, scale, ws=None, ws_bytes=0, fill=None,
+                     stream=None):
+    sp, spp = _i32(spans)
+    sk, skp = _i32(sinks)
+    _check(load().moa_prefill_sink(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, Hq, Hkv, int(N), d, _dtype(dtype), spp,
+                                   skp, float(scale), _ptr(ws), ws_bytes, fill, _stream(stream)), "moa_prefill_sink")
+
+
+def moa_workspace_bytes_sink(op, B, Hq, N, d, spans, sinks):
+    sp, spp = _i32(spans)
+    sk, skp = _i32(sinks)
+    out = ctypes.c_size_t()
+    _check(load().moa_workspace_bytes_sink(op, B, Hq, int(N), d, spp, skp, ctypes.byref(out)),
+           "moa_workspace_bytes_sink")
+    return out.value
+
+
+def moa_decode_sink(handle, q, o, Hq, spans, sinks, scale, ws, ws_bytes, stream=None):
+    sp, spp = _i32(spans)
+    sk, skp = _i32(sinks)
+    _check(load().moa_decode_sink(handle, _ptr(q), _ptr(o), Hq, spp, skp, float(scale), _ptr(ws), ws_bytes,
+                                  _stream(stream)), "moa_decode_sink")
+
+
+def moa_decode_append_sink(handle, q, k, v, o, Hq, spans, sinks, scale, ws, ws_bytes, stream=None):
+    sp, spp = _i32(spans)
+    sk, skp = _i32(sinks)
+    _check(load().moa_decode_append_sink(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), Hq, spp, skp, float(scale),
+                                         _ptr(ws), ws_bytes, _stream(stream)), "moa_decode_append_sink")
+
+
 # ---- conveniences over torch-owned device memory ------------------------------
 class KVCache:
     """A ring-buffer cache whose device buffer is a torch uint8 tensor."""
 
-    def __init__(self, B, Hkv, d, dtype, capacity, device="cuda", stream=None):
+    def __init__(self, B, Hkv, d, dtype, capacity, device="cuda", stream=None, sink_capacity=None):
         import torch
         self.B, self.Hkv, self.d, self.dtype = B, Hkv, d, _dtype(dtype)
         self.capacity = [int(c) for c in capacity]
-        self.nbytes = moa_kv_bytes(B, Hkv, d, self.dtype, self.capacity)
+        self.sink_capacity = None if sink_capacity is None else [int(c) for c in sink_capacity]
+        if self.sink_capacity is None:
+            self.nbytes = moa_kv_bytes(B, Hkv, d, self.dtype, self.capacity)
+        else:
+            self.nbytes = moa_kv_bytes_sink(B, Hkv, d, self.dtype, self.capacity, self.sink_capacity)
         self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
         base = self.buf.data_ptr()
         self.ptr = (base + 255) // 256 * 256
-        self.handle = moa_kv_alloc(self.ptr, self.nbytes, B, Hkv, d, self.dtype, self.capacity, stream)
+        if self.sink_capacity is None:
+            self.handle = moa_kv_alloc(self.ptr, self.nbytes, B, Hkv, d, self.dtype, self.capacity, stream)
+        else:
+            self.handle = moa_kv_alloc_sink(self.ptr, self.nbytes, B, Hkv, d, self.dtype, self.capacity,
+                                            self.sink_capacity, stream)
 
     def append(self, k, v, stream=None):
         moa_kv_append(self.handle, k, v, k.shape[2], stream)

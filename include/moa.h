@@ -267,6 +267,71 @@ moa_status moa_decode_append(moa_kv_cache* cache, const void* q, const void* k, 
                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Band plus global ("sink") tokens.  The codewithpapers page for arXiv
+ * 2406.14909 lists, from the official repository, a global-pattern generator
+ * (gen_global_pattern) beside the band pattern and StreamingLLM density
+ * counters; the project page's Table 4 compares with StreamingLLM.  The pages
+ * give no formula; the reading taken: query head h keeps its band and, in
+ * addition, attends to the first k_h positions of the sequence (those that
+ * are causal), each key once:
+ *   keys(i) = { j : i - S_h < j <= i }  union  { j : 0 <= j < k_h, j <= i }.
+ * k_h = 0 for every head gives exactly the plain entry points above.
+ *
+ * A cache that serves such heads keeps, besides the ring, the first K_g
+ * positions of every sequence for good: sink_capacity[g] = K_g >= the k_h of
+ * every query head of key/value head g.  Layout: the plain layout above
+ * (header, ring region), then the global-token region: for b in [0,B), for g
+ * in [0,Hkv): K rows [K_g][d], then V rows [K_g][d]; position p < K_g at row
+ * p.  Its block for (b, g) starts at element
+ * (b * sum_g K_g + sum_{g'<g} K_g') * 2 * d of the region, which starts at
+ * byte H + B * sum_g C_g * 2 * d * elem_size.  Every append (moa_kv_append,
+ * the prefill fill, the fused decode append, the chunked prefill) also writes
+ * positions below K_g there.  sum_g K_g <= 2^31 - 1.
+ * ------------------------------------------------------------------------- */
+
+/* moa_kv_bytes / moa_kv_alloc for a cache with global-token rows.
+ * sink_capacity: host int32[Hkv], each >= 0 (NULL = all 0, the plain cache). */
+moa_status moa_kv_bytes_sink(int32_t B, int32_t Hkv, int32_t d, moa_dtype dtype,
+                             const int32_t* capacity, const int32_t* sink_capacity,
+                             size_t* bytes_out);
+moa_status moa_kv_alloc_sink(void* dev_buf, size_t bytes, int32_t B, int32_t Hkv, int32_t d,
+                             moa_dtype dtype, const int32_t* capacity,
+                             const int32_t* sink_capacity, void* stream, moa_kv_cache** out);
+
+/* moa_prefill with global tokens: sinks is host int32[Hq], each >= 0 (values
+ * above N behave as N).  With fill_or_null, sinks[h] <= K_{h/(Hq/Hkv)} of the
+ * cache (else MOA_ERR_CAPACITY).  Same kernels, launches, workspace and errors
+ * as moa_prefill: the tensor-core kernel adds to each query tile's band the
+ * key tiles that hold its global tokens. */
+moa_status moa_prefill_sink(const void* q, const void* k, const void* v, void* o,
+                            int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
+                            moa_dtype dtype, const int32_t* spans, const int32_t* sinks,
+                            float scale, void* workspace, size_t ws_bytes,
+                            moa_kv_cache* fill_or_null, void* stream);
+
+/* Decode workspace size with global tokens (sinks: host int32[Hq], >= 0);
+ * for MOA_OP_PREFILL it equals moa_workspace_bytes. */
+moa_status moa_workspace_bytes_sink(moa_op op, int32_t B, int32_t Hq, int64_t N, int32_t d,
+                                    const int32_t* spans, const int32_t* sinks,
+                                    size_t* bytes_out);
+
+/* moa_decode / moa_decode_append with global tokens: the query at position
+ * t = t_b - 1 of head h attends to keys(t) above, its band through the ring
+ * and the global tokens below the band from the global-token rows.
+ * sinks: host int32[Hq], 0 <= sinks[h] <= K_{h/(Hq/Hkv)} (else
+ * MOA_ERR_CAPACITY).  workspace: moa_workspace_bytes_sink(MOA_OP_DECODE, ...)
+ * bytes, zeroed before first use.  One launch: the per-head split-KV kernel,
+ * with ceil(k_h / 512) more splits per head over the global-token rows (the
+ * group-shared kernels do not take global tokens).  Errors as moa_decode. */
+moa_status moa_decode_sink(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
+                           const int32_t* spans, const int32_t* sinks, float scale,
+                           void* workspace, size_t ws_bytes, void* stream);
+moa_status moa_decode_append_sink(moa_kv_cache* cache, const void* q, const void* k,
+                                  const void* v, void* o, int32_t Hq, const int32_t* spans,
+                                  const int32_t* sinks, float scale, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Decode without a caller workspace.  The paper has no counterpart: this is
  * a deployment convenience of this library.
  *

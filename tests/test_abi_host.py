@@ -280,3 +280,40 @@ def test_input_tables_reach_target_density():
     spans = orules.eval_spans(a, b, 16384, 64)
     assert abs(np.mean(spans) / 16384 - 0.5) < 0.05
     assert set(np.unique(b)) <= {0.0, 0.5, 0.9}
+
+
+def test_sink_cache_sizes_and_errors():
+    for B, Hkv, d, caps, sinks, dt, eb in [(2, 2, 64, [3, 2], [2, 1], "f32", 4),
+                                          (3, 4, 128, [5, 1, 9, 4], [0, 0, 7, 0], "bf16", 2),
+                                          (1, 1, 128, [8], [0], "bf16", 2)]:
+        assert moa.moa_kv_bytes_sink(B, Hkv, d, dt, caps, sinks) == okv.buffer_bytes(B, Hkv, d, caps, eb, sinks)
+    assert moa.moa_kv_bytes_sink(2, 2, 128, "bf16", [3, 5], [0, 0]) == moa.moa_kv_bytes(2, 2, 128, "bf16", [3, 5])
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_kv_bytes_sink(1, 2, 128, "bf16", [4, 4], [1, -1])     # negative global-token rows
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_kv_bytes_sink(1, 2, 128, "bf16", [4, 4], [1 << 30, 1 << 30])   # sum above 2^31 - 1
+    assert e.value.status == moa.MOA_ERR_INVALID_ARG
+
+
+def test_sink_prefill_and_workspace_argument_errors_need_no_gpu():
+    ok = dict(q=4096, k=4096, v=4096, o=4096, B=1, Hq=4, Hkv=2, N=256, d=128, dtype="bf16",
+              spans=[64] * 4, sinks=[4] * 4, scale=0.088, ws=None, ws_bytes=0, stream=0)
+    for change, status in [(dict(sinks=[4, -1, 0, 0]), moa.MOA_ERR_INVALID_ARG),
+                           (dict(spans=[0, 1, 1, 1]), moa.MOA_ERR_INVALID_ARG),
+                           (dict(), moa.MOA_ERR_WORKSPACE)]:
+        args = dict(ok)
+        args.update(change)
+        with pytest.raises(moa.MoaError) as e:
+            moa.moa_prefill_sink(**args)
+        assert e.value.status == status, change
+    spans, sinks = [64, 300, 4096, 1], [0, 600, 4, 1]
+    plain = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans)
+    more = moa.moa_workspace_bytes_sink(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans, sinks)
+    assert more > plain and more % 256 == 0
+    assert moa.moa_workspace_bytes_sink(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans, [0] * 4) == plain
+    assert moa.moa_workspace_bytes_sink(moa.MOA_OP_PREFILL, 2, 4, 1000, 128, spans, sinks) == \
+        moa.moa_workspace_bytes(moa.MOA_OP_PREFILL, 2, 4, 1000, 128, spans)
+    with pytest.raises(moa.MoaError):
+        moa.moa_workspace_bytes_sink(moa.MOA_OP_DECODE, 2, 4, 0, 128, spans, [0, -2, 0, 0])
+
