@@ -29,6 +29,11 @@ namespace {
 constexpr int kDecThreads = 128;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kChunk = 512;          // window entries per split
+#ifndef MOA_GQA_CHUNK
+#define MOA_GQA_CHUNK 512
+#endif
+constexpr int kGroupChunk = MOA_GQA_CHUNK;   // group-window entries per split of the group kernels
+static_assert(kGroupChunk >= kChunk && kGroupChunk % kChunk == 0, "group split size");
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
 #ifndef MOA_GROUP_MMA
 #define MOA_GROUP_MMA 1
@@ -358,8 +363,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);   // the group's longest window
-  const int w0 = s * kChunk;
-  const int nrows = max(0, min(kChunk, W - w0));
+  const int w0 = s * kGroupChunk;
+  const int nrows = max(0, min(kGroupChunk, W - w0));
   const int64_t pos0 = tb - W + w0;
   const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
 
@@ -594,7 +599,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
 // Grouped-query decode on the tensor cores (bf16, d = 128).
 //
 // Same work item, window geometry and partial layout as decode_group_kernel:
-// one CTA per (b, KV group g, split of kChunk group-window entries).  Warp w
+// one CTA per (b, KV group g, split of kGroupChunk group-window entries).  Warp w
 // takes entries [128w, 128w + 128) of the split in tiles of 16 cached rows:
 //   * cp.async copies the tile's K and V rows (16 x 256 bytes each) into a
 //     two-stage per-warp buffer, 16-byte chunks XOR-swizzled by row so that
@@ -613,8 +618,12 @@ constexpr int kMmaTileBytes = kMmaRows * 128 * 2; // one 16 x 128 bf16 tile
 #define MOA_MMA_STAGES 2
 #endif
 constexpr int kMmaStages = MOA_MMA_STAGES;        // K/V tiles in flight per warp + 1
+#ifndef MOA_GQA_SPLIT_ACC
+#define MOA_GQA_SPLIT_ACC 0
+#endif
+constexpr bool kGroupSplitAcc = MOA_GQA_SPLIT_ACC != 0;
 constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
-constexpr int kMmaWarpRows = kChunk / kDecWarps;  // entries per warp and split
+constexpr int kMmaWarpRows = kGroupChunk / kDecWarps;  // entries per warp and split
 constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -670,8 +679,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;
   const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);
-  const int w0 = s * kChunk;
-  const int nrows = max(0, min(kChunk, W - w0));
+  const int w0 = s * kGroupChunk;
+  const int nrows = max(0, min(kGroupChunk, W - w0));
   const int64_t pos0 = tb - W + w0;
   const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
   const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
@@ -764,16 +773,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     cp_async_wait<kMmaStages - 1>();                    // tile ti has landed
     __syncwarp();
     const uint32_t tK = sbase + (uint32_t)(ti % kMmaStages) * 2 * kMmaTileBytes, tV = tK + kMmaTileBytes;
-    // S^T = K . Q^T
+    // S^T = K . Q^T (two accumulators: two independent MMA chains)
     float sacc[4] = {0.f, 0.f, 0.f, 0.f};
     {
+      float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
       const int ar = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t a[4];
         ldsm_x4(tK + swz(ar, 2 * kk + (lane >> 4)), a);
-        mma16816(sacc, a, qb[kk][0], qb[kk][1]);
+        mma16816((kk & 1) && kGroupSplitAcc ? sacc2 : sacc, a, qb[kk][0], qb[kk][1]);
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
     }
     // mask and scale: rows g4 and g4 + 8 of the tile, heads h0 and h1
     const int ra = wrow0 + ti * kMmaRows + g4, rb = ra + 8;
@@ -1041,7 +1053,7 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
     p.split_pre[0] = 0;
     p.hslot_pre[0] = 0;
     for (int g = 0; g < c->Hkv; ++g) {
-      const int ns = (c->cap[g] + kChunk - 1) / kChunk;
+      const int ns = (c->cap[g] + kGroupChunk - 1) / kGroupChunk;
       p.split_pre[g + 1] = p.split_pre[g] + ns;
       for (int j = 0; j < G; ++j) p.hslot_pre[g * G + j + 1] = p.hslot_pre[g * G + j] + ns;
       items += ns;

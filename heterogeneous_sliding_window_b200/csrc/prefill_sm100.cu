@@ -76,8 +76,18 @@ constexpr int kD = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one 128 x 128 bf16 tile
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizzled half
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
-constexpr uint32_t kQSlots = 3;                       // rotating Q tiles (two per unit)
-constexpr uint32_t kKStages = 2, kVStages = 2;        // K and V ring depths
+// Ring depths (compile-time choices; shared memory holds seven 32 KB tiles).
+#ifndef MOA_PREFILL_Q_SLOTS
+#define MOA_PREFILL_Q_SLOTS 3
+#endif
+#ifndef MOA_PREFILL_K_STAGES
+#define MOA_PREFILL_K_STAGES 2
+#endif
+#ifndef MOA_PREFILL_V_STAGES
+#define MOA_PREFILL_V_STAGES 2
+#endif
+constexpr uint32_t kQSlots = MOA_PREFILL_Q_SLOTS;     // rotating Q tiles (two per unit)
+constexpr uint32_t kKStages = MOA_PREFILL_K_STAGES, kVStages = MOA_PREFILL_V_STAGES;   // K and V ring depths
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + kQSlots * kTileBytes;
 constexpr uint32_t OFF_V = OFF_K + kKStages * kTileBytes;
@@ -100,7 +110,8 @@ enum {
   B_KFULL0 = B_UEMPTY0 + 4, B_KEMPTY0 = B_KFULL0 + 4, B_VFULL0 = B_KEMPTY0 + 4, B_VEMPTY0 = B_VFULL0 + 4,
   B_COUNT = B_VEMPTY0 + 4
 };
-static_assert(kQSlots == 3 && kKStages <= 4 && kVStages <= 4, "ring depth");
+static_assert(kQSlots >= 2 && kQSlots <= 3 && kKStages >= 2 && kKStages <= 4 && kVStages >= 2 && kVStages <= 4,
+              "ring depth");
 constexpr uint32_t OFF_TMEM_SLOT = OFF_BAR + 8 * B_COUNT;        // uint32
 constexpr uint32_t OFF_ABORT = OFF_TMEM_SLOT + 4;                // int
 constexpr uint32_t kUnitSlots = 4;                                // unit record ring depth
