@@ -622,6 +622,9 @@ constexpr int kMmaStages = MOA_MMA_STAGES;        // K/V tiles in flight per war
 #define MOA_GQA_SPLIT_ACC 0
 #endif
 constexpr bool kGroupSplitAcc = MOA_GQA_SPLIT_ACC != 0;
+#ifndef MOA_GQA_FAST_ADDR
+#define MOA_GQA_FAST_ADDR 0
+#endif
 constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
 constexpr int kMmaWarpRows = kGroupChunk / kDecWarps;  // entries per warp and split
 constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
@@ -719,6 +722,43 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   const int ntiles = (wrows + kMmaRows - 1) / kMmaRows;
 
   // issue the copies of tile ti into stage st (rows past the split are zero-filled)
+#if MOA_GQA_FAST_ADDR
+  // Lane `lane` copies chunk cc = lane & 15 of tile rows rr0 + 2q, q = 0..7
+  // (rr0 = lane >> 4): its slot advances by 2 per row with one wrap test, and
+  // its swizzled destinations repeat every four rows (row residues mod 8 are
+  // rr0 + 2(q & 3)), so they are computed once.
+  const int cc = lane & 15, rr0 = lane >> 4;
+  uint32_t soff[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) soff[u] = swz(rr0 + 2 * u, cc);
+  auto load_tile = [&](int ti, int st) {
+    const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
+    int row = wrow0 + ti * kMmaRows + rr0;                       // split entry of q = 0
+    int slot = slot0 + row;
+    if (slot >= C) slot -= C;                                    // exact while row < nrows <= C
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const bool ok = row < nrows;
+      const __nv_bfloat16* srcK = ok ? Kb + (size_t)slot * D + cc * 8 : Kb;
+      const __nv_bfloat16* srcV = ok ? Vb + (size_t)slot * D + cc * 8 : Vb;
+      if (ok && w0 + row == e_new) {
+        // this CTA is the group's only reader of the newest entry: write it to its slot
+        const int4 kx = __ldg(reinterpret_cast<const int4*>(kn + cc * 8));
+        const int4 vx = __ldg(reinterpret_cast<const int4*>(vn + cc * 8));
+        *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(srcK)) = kx;
+        *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(srcV)) = vx;
+        srcK = kn + cc * 8;
+        srcV = vn + cc * 8;
+      }
+      const uint32_t off = (uint32_t)(q >> 2) * 2048u + soff[q & 3];
+      cp_async16(dK + off, srcK, ok ? 16u : 0u);
+      cp_async16(dV + off, srcV, ok ? 16u : 0u);
+      row += 2;
+      slot += 2;
+      if (slot >= C) slot -= C;
+    }
+  };
+#else
   auto load_tile = [&](int ti, int st) {
     const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
 #pragma unroll
@@ -752,6 +792,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
       cp_async16(dV + swz(rr, cc), srcV, bytes);
     }
   };
+#endif
 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h1
   float oacc[8][4];
