@@ -86,6 +86,10 @@ constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizz
 #ifndef MOA_PREFILL_V_STAGES
 #define MOA_PREFILL_V_STAGES 2
 #endif
+#ifndef MOA_PREFILL_EARLY_SB
+#define MOA_PREFILL_EARLY_SB 0
+#endif
+constexpr bool kEarlySB = MOA_PREFILL_EARLY_SB != 0;   // tile B's first S issued in the unit's prologue
 constexpr uint32_t kQSlots = MOA_PREFILL_Q_SLOTS;     // rotating Q tiles (two per unit)
 constexpr uint32_t kKStages = MOA_PREFILL_K_STAGES, kVStages = MOA_PREFILL_V_STAGES;   // K and V ring depths
 constexpr uint32_t OFF_Q = 0;
@@ -553,6 +557,21 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
     }
     mma_commit(c.bar(B_KEMPTY0 + kst));
     if (++kst == kKStages) { kst = 0; kph ^= 1u; }
+    // When tile B starts one stream tile after tile A, its first S goes to
+    // the tensor core now rather than after PV_A of the first tile, so B's
+    // softmax can work while A's finishes the previous unit's epilogue.  The
+    // ring's next K slot holds that tile; it is released in the loop as usual.
+    bool sB_early = false;
+    if (kEarlySB && x.hasB && x.start < x.R && !x.in(1, x.start) && x.first[1] == x.next(x.start)) {
+      if (!c.wait(B_KFULL0 + kst, kph)) return;
+      if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
+      qrB = true;
+      tc_fence_after();
+      mma_qk(tSB, desc_qk_lo(sQ0 + q.sB * kTileBytes), desc_qk_lo(sK0 + kst * kTileBytes), hi);
+      mma_commit(c.bar(B_SFULL0 + 1));
+      if (x.first[1] == x.m[1]) mma_commit(c.bar(B_QEMPTY0 + q.sB));
+      sB_early = true;
+    }
     // next unit, when its tile A could start during this unit's last step
     bool have_next = false, ended = false;
     int4 Uy = make_int4(0, 0, 0, 0);
@@ -617,7 +636,7 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
             ++ucB;
           }
         }
-        if (more && x.in(1, jn)) {
+        if (more && x.in(1, jn) && !(sB_early && j == x.start)) {
           if (!qrB) {
             if (!c.wait(B_QFULL0 + q.sB, q.pB)) return;
             qrB = true;
