@@ -42,6 +42,10 @@ constexpr int kChunk = MOA_DECODE_CHUNK;   // window entries per split (per-head
 constexpr int kGroupChunk = MOA_GQA_CHUNK;
 static_assert(kGroupChunk >= kChunk && kGroupChunk % kChunk == 0, "group split size");
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
+#ifndef MOA_DECODE_PAIRS
+#define MOA_DECODE_PAIRS 0
+#endif
+constexpr bool kDecodePairs = MOA_DECODE_PAIRS != 0;   // packed f32x2 FMAs in the per-head kernel
 #ifndef MOA_GROUP_MMA
 #define MOA_GROUP_MMA 1
 #endif
@@ -232,8 +236,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       float kf[VE];
       Vec16<T>::cvt(kr[u], kf);
       float dot = 0.f;
+      if constexpr (kDecodePairs) {
+        uint64_t d2 = 0;
 #pragma unroll
-      for (int e = 0; e < VE; ++e) dot = fmaf(qf[e], kf[e], dot);
+        for (int e = 0; e < VE / 2; ++e) d2 = sm100::f2_fma(sm100::f2_pack(qf[2 * e], qf[2 * e + 1]),
+                                                          sm100::f2_pack(kf[2 * e], kf[2 * e + 1]), d2);
+        float d0, d1;
+        sm100::f2_unpack(d2, d0, d1);
+        dot = d0 + d1;
+      } else {
+#pragma unroll
+        for (int e = 0; e < VE; ++e) dot = fmaf(qf[e], kf[e], dot);
+      }
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       sv[u] = (base + u * NG + grp < nrows) ? dot : -INFINITY;
@@ -255,8 +269,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       l += pu;
       float vf[VE];
       Vec16<T>::cvt(vr[u], vf);
+      if constexpr (kDecodePairs) {
+        const uint64_t p2 = sm100::f2_pack(pu, pu);
 #pragma unroll
-      for (int e = 0; e < VE; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
+        for (int e = 0; e < VE / 2; ++e) {
+          const uint64_t a2 = sm100::f2_fma(p2, sm100::f2_pack(vf[2 * e], vf[2 * e + 1]),
+                                            sm100::f2_pack(acc[2 * e], acc[2 * e + 1]));
+          sm100::f2_unpack(a2, acc[2 * e], acc[2 * e + 1]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < VE; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
+      }
     }
   }
 
@@ -635,6 +659,12 @@ constexpr bool kGroupSplitAcc = MOA_GQA_SPLIT_ACC != 0;
 #ifndef MOA_GQA_FAST_ADDR
 #define MOA_GQA_FAST_ADDR 1
 #endif
+// ... and the copies of a tile whose 16 slots are contiguous from one base
+// pointer with constant offsets (1), or always the per-copy walk (0).
+#ifndef MOA_GQA_TILE_FAST
+#define MOA_GQA_TILE_FAST 1
+#endif
+constexpr bool kGroupTileFast = MOA_GQA_TILE_FAST != 0;
 constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
 constexpr int kMmaWarpRows = kGroupChunk / kDecWarps;  // entries per warp and split
 constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
@@ -741,9 +771,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   uint32_t soff[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) soff[u] = swz(rr0 + 2 * u, cc);
+  const size_t vofs = (size_t)C * D;                           // V block after the K block
   auto load_tile = [&](int ti, int st) {
     const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
-    int row = wrow0 + ti * kMmaRows + rr0;                       // split entry of q = 0
+    const int trow = wrow0 + ti * kMmaRows;                      // the tile's first split entry
+    int tslot = slot0 + trow;
+    if (tslot >= C) tslot -= C;
+    // Common case: all 16 rows inside the split, their slots contiguous (no
+    // wrap), none the fused append's new entry: one base pointer per lane and
+    // constant offsets (two rows, 512 bytes, apart per copy).
+    if (kGroupTileFast && trow + kMmaRows <= nrows && tslot + kMmaRows <= C &&
+        !(e_new >= w0 + trow && e_new < w0 + trow + kMmaRows)) {
+      const __nv_bfloat16* pk = Kb + (size_t)(tslot + rr0) * D + cc * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t off = (uint32_t)(q >> 2) * 2048u + soff[q & 3];
+        cp_async16(dK + off, pk + (size_t)q * 2 * D, 16u);
+        cp_async16(dV + off, pk + vofs + (size_t)q * 2 * D, 16u);
+      }
+      return;
+    }
+    int row = trow + rr0;                                        // split entry of q = 0
     int slot = slot0 + row;
     if (slot >= C) slot -= C;                                    // exact while row < nrows <= C
 #pragma unroll

@@ -18,9 +18,10 @@
 //    so far, so heads with very different spans balance across SMs without
 //    atomics and every CTA can read its next units ahead of time.
 //  * Warp roles (384 threads, setmaxnreg split 120 / 192 / 192):
-//      warp 0       TMA producer: the unit's two Q tiles into three rotating
-//                   Q slots (the next unit's Q loads while this unit runs),
-//                   K and V tiles through two-stage rings (128-byte swizzle).
+//      warp 0       TMA producer: the unit's two Q tiles into two rotating
+//                   Q slots (the next unit's Q_A loads once this unit's A is
+//                   done), K tiles through a three-stage ring and V tiles
+//                   through a two-stage ring (128-byte swizzle).
 //      warp 1       MMA issuer (one thread), tcgen05.mma M=128, N=128, K=16.
 //                   Per key tile j:  O_A += P_A(j) V(j),  S_A(j+1) = Q_A K(j+1)^T,
 //                   O_B += P_B(j) V(j),  S_B(j+1) = Q_B K(j+1)^T.
@@ -77,17 +78,21 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one 128 x 128 bf16 tile
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;    // one 128-row x 128-byte swizzled half
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
 // Ring depths (compile-time choices; shared memory holds seven 32 KB tiles).
+// Two Q slots and three K stages measured best on the Vicuna-7B-shaped prompt
+// (25 % density, with the early first S of tile B: 885 against 857 TFLOP/s
+// back to back for three Q slots and two K stages, 839-846 against 772-826
+// after an L2 flush).
 #ifndef MOA_PREFILL_Q_SLOTS
-#define MOA_PREFILL_Q_SLOTS 3
+#define MOA_PREFILL_Q_SLOTS 2
 #endif
 #ifndef MOA_PREFILL_K_STAGES
-#define MOA_PREFILL_K_STAGES 2
+#define MOA_PREFILL_K_STAGES 3
 #endif
 #ifndef MOA_PREFILL_V_STAGES
 #define MOA_PREFILL_V_STAGES 2
 #endif
 #ifndef MOA_PREFILL_EARLY_SB
-#define MOA_PREFILL_EARLY_SB 0
+#define MOA_PREFILL_EARLY_SB 1
 #endif
 constexpr bool kEarlySB = MOA_PREFILL_EARLY_SB != 0;   // tile B's first S issued in the unit's prologue
 constexpr uint32_t kQSlots = MOA_PREFILL_Q_SLOTS;     // rotating Q tiles (two per unit)
