@@ -338,7 +338,10 @@ __device__ __forceinline__ float max64(const float* s) {
 // than by MUFU ex2: one in kPolyEvery.  MUFU issues 16 ex2 per clock per SM,
 // which equals the tensor core's pace at d = 128, so moving part of the work
 // to the FMA pipe shortens the softmax, the critical path between two MMAs.
-constexpr int kPolyEvery = 8;
+#ifndef MOA_PREFILL_POLY_EVERY
+#define MOA_PREFILL_POLY_EVERY 8
+#endif
+constexpr int kPolyEvery = MOA_PREFILL_POLY_EVERY;
 
 // p = 2^(s * c - m) for 64 scores as bf16 pairs w[32]; returns the fp32 sum.
 __device__ __forceinline__ float exp_half(const float* s, float c, float neg, uint32_t* w) {
