@@ -726,13 +726,36 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;
   const int W = (int)(tb < (int64_t)C ? tb : (int64_t)C);
-  const int w0 = s * kGroupChunk;
-  const int nrows = max(0, min(kGroupChunk, W - w0));
+  // Splits s >= nwin cover the group's global tokens below its heads' windows:
+  // positions 0 .. GW - 1 (the union over the group's heads), rows of the
+  // global-token region, which do not wrap.
+  const int nwin = (C + kGroupChunk - 1) / kGroupChunk;
+  const bool gsplit = s >= nwin;
+  int GW = 0;
+  if (gsplit) {
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      const int64_t Sj = tb < (int64_t)p.span[g * G + j] ? tb : (int64_t)p.span[g * G + j];
+      GW = max(GW, (int)min((int64_t)p.sink[g * G + j], tb - Sj));
+    }
+  }
+  const int w0 = (gsplit ? s - nwin : s) * kGroupChunk;
+  const int nrows = max(0, min(kGroupChunk, (gsplit ? GW : W) - w0));
   const int64_t pos0 = tb - W + w0;
-  const int slot0 = nrows > 0 ? (int)(pos0 % C) : 0;
+  const int slot0 = gsplit ? w0 : nrows > 0 ? (int)(pos0 % C) : 0;
+  const int Cw = gsplit ? (1 << 30) : C;           // global-token rows do not wrap
   const __nv_bfloat16* Kb = reinterpret_cast<const __nv_bfloat16*>(p.data) + (size_t)((int64_t)b * p.sumC + p.goff[g]) * 2 * D;
   const __nv_bfloat16* Vb = Kb + (size_t)C * D;
-  const int e_new = fused ? W - 1 : -1;
+  if (gsplit) {
+    Kb = reinterpret_cast<const __nv_bfloat16*>(p.sink_data) + (size_t)((int64_t)b * p.sumK + p.soff[g]) * 2 * D;
+    Vb = Kb + (size_t)p.scap[g] * D;
+  }
+  const int e_new = fused && !gsplit ? W - 1 : -1;
+  // the fused append also keeps the new token's global-token row
+  __nv_bfloat16* ks_new = nullptr;
+  if (fused && !gsplit && p.sink_data != nullptr && t0 < (int64_t)p.scap[g])
+    ks_new = reinterpret_cast<__nv_bfloat16*>(p.sink_data) + (size_t)((int64_t)b * p.sumK + p.soff[g]) * 2 * D +
+             (size_t)t0 * D;
   const __nv_bfloat16* kn = fused ? reinterpret_cast<const __nv_bfloat16*>(p.k_new) + ((size_t)b * Hkv + g) * D : nullptr;
   const __nv_bfloat16* vn = fused ? reinterpret_cast<const __nv_bfloat16*>(p.v_new) + ((size_t)b * Hkv + g) * D : nullptr;
 
@@ -748,14 +771,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
       qb[kk][1] = hv ? __ldg(qrow + 8 * kk + c4 + 4) : 0u;
     }
   }
-  // heads this lane owns in the accumulator layouts, and where their windows start
+  // heads this lane owns in the accumulator layouts, and the entries [e0, e1)
+  // of this split's range each head sees (window splits: from where its window
+  // starts; global splits: below the end of its global tokens)
   const int h0 = 2 * c4, h1 = 2 * c4 + 1;
   int e0a = 1 << 30, e0b = 1 << 30;              // past every entry: heads beyond G see no row
+  int e1a = 1 << 30, e1b = 1 << 30;
 #pragma unroll
   for (int j = 0; j < G; ++j) {
     const int Sh = (int)(tb < (int64_t)p.span[g * G + j] ? tb : (int64_t)p.span[g * G + j]);
-    if (j == h0) e0a = W - Sh;
-    if (j == h1) e0b = W - Sh;
+    const int lo_j = gsplit ? 0 : W - Sh;
+    const int hi_j = gsplit ? (int)min((int64_t)p.sink[g * G + j], tb - Sh) : (1 << 30);
+    if (j == h0) { e0a = lo_j; e1a = hi_j; }
+    if (j == h1) { e0b = lo_j; e1b = hi_j; }
   }
 
   const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(dsm) + (uint32_t)warp * kMmaWarpBytes;
@@ -775,16 +803,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   uint32_t soff[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) soff[u] = swz(rr0 + 2 * u, cc);
-  const size_t vofs = (size_t)C * D;                           // V block after the K block
+  const size_t vofs = (size_t)(Vb - Kb);                       // V block after the K block
   auto load_tile = [&](int ti, int st) {
     const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
     const int trow = wrow0 + ti * kMmaRows;                      // the tile's first split entry
     int tslot = slot0 + trow;
-    if (tslot >= C) tslot -= C;
+    if (tslot >= Cw) tslot -= Cw;
     // Common case: all 16 rows inside the split, their slots contiguous (no
     // wrap), none the fused append's new entry: one base pointer per lane and
     // constant offsets (two rows, 512 bytes, apart per copy).
-    if (kGroupTileFast && trow + kMmaRows <= nrows && tslot + kMmaRows <= C &&
+    if (kGroupTileFast && trow + kMmaRows <= nrows && tslot + kMmaRows <= Cw &&
         !(e_new >= w0 + trow && e_new < w0 + trow + kMmaRows)) {
       const __nv_bfloat16* pk = Kb + (size_t)(tslot + rr0) * D + cc * 8;
 #pragma unroll
@@ -797,7 +825,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     }
     int row = trow + rr0;                                        // split entry of q = 0
     int slot = slot0 + row;
-    if (slot >= C) slot -= C;                                    // exact while row < nrows <= C
+    if (slot >= Cw) slot -= Cw;                                  // exact while row < nrows <= C
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const bool ok = row < nrows;
@@ -809,6 +837,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
         const int4 vx = __ldg(reinterpret_cast<const int4*>(vn + cc * 8));
         *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(srcK)) = kx;
         *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(srcV)) = vx;
+        if (ks_new != nullptr) {
+          *reinterpret_cast<int4*>(ks_new + cc * 8) = kx;
+          *reinterpret_cast<int4*>(ks_new + (size_t)p.scap[g] * D + cc * 8) = vx;
+        }
         srcK = kn + cc * 8;
         srcV = vn + cc * 8;
       }
@@ -817,7 +849,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
       cp_async16(dV + off, srcV, ok ? 16u : 0u);
       row += 2;
       slot += 2;
-      if (slot >= C) slot -= C;
+      if (slot >= Cw) slot -= Cw;
     }
   };
 #else
@@ -837,15 +869,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
           srcK = kn + cc * 8;
           srcV = vn + cc * 8;
           int slot = slot0 + row;
-          if (slot >= C) slot -= C;
+          if (slot >= Cw) slot -= Cw;
           // this CTA is the group's only reader of the newest entry: write it to its slot
-          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Kb) + (size_t)slot * D + cc * 8) =
-              __ldg(reinterpret_cast<const int4*>(srcK));
-          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Vb) + (size_t)slot * D + cc * 8) =
-              __ldg(reinterpret_cast<const int4*>(srcV));
+          const int4 kx = __ldg(reinterpret_cast<const int4*>(srcK));
+          const int4 vx = __ldg(reinterpret_cast<const int4*>(srcV));
+          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Kb) + (size_t)slot * D + cc * 8) = kx;
+          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Vb) + (size_t)slot * D + cc * 8) = vx;
+          if (ks_new != nullptr) {
+            *reinterpret_cast<int4*>(ks_new + cc * 8) = kx;
+            *reinterpret_cast<int4*>(ks_new + (size_t)p.scap[g] * D + cc * 8) = vx;
+          }
         } else {
           int slot = slot0 + row;
-          if (slot >= C) slot -= C;
+          if (slot >= Cw) slot -= Cw;
           srcK = Kb + (size_t)slot * D + cc * 8;
           srcV = Vb + (size_t)slot * D + cc * 8;
         }
@@ -893,10 +929,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     // mask and scale: rows g4 and g4 + 8 of the tile, heads h0 and h1
     const int ra = wrow0 + ti * kMmaRows + g4, rb = ra + 8;
     const float sc = p.scale_log2;
-    const float s0 = (ra < nrows && w0 + ra >= e0a) ? sacc[0] * sc : -INFINITY;
-    const float s1 = (ra < nrows && w0 + ra >= e0b) ? sacc[1] * sc : -INFINITY;
-    const float s2 = (rb < nrows && w0 + rb >= e0a) ? sacc[2] * sc : -INFINITY;
-    const float s3 = (rb < nrows && w0 + rb >= e0b) ? sacc[3] * sc : -INFINITY;
+    const float s0 = (ra < nrows && w0 + ra >= e0a && w0 + ra < e1a) ? sacc[0] * sc : -INFINITY;
+    const float s1 = (ra < nrows && w0 + ra >= e0b && w0 + ra < e1b) ? sacc[1] * sc : -INFINITY;
+    const float s2 = (rb < nrows && w0 + rb >= e0a && w0 + rb < e1a) ? sacc[2] * sc : -INFINITY;
+    const float s3 = (rb < nrows && w0 + rb >= e0b && w0 + rb < e1b) ? sacc[3] * sc : -INFINITY;
     float t0m = fmaxf(s0, s2), t1m = fmaxf(s1, s3);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -1148,18 +1184,22 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   int64_t head_rows = 0, group_rows = 0;
   for (int h = 0; h < Hq; ++h) head_rows += spans[h];
   for (int g = 0; g < c->Hkv; ++g) group_rows += c->cap[g];
-  // Global tokens, and any cache that keeps global-token rows (the fused
-  // append writes them), take the per-head kernel.
+  // The tensor-core group kernel also serves global tokens (splits over the
+  // group's global-token rows) and keeps the rows of caches that hold them.
+  // The SIMT group kernel does neither: such calls take the per-head kernel.
   const bool plain = p.sink_data == nullptr;
-  const bool mma_group = plain && kGroupMma && c->dtype == MOA_BF16 && c->d == 128 &&
+  const bool mma_group = kGroupMma && c->dtype == MOA_BF16 && c->d == 128 &&
                          (G == 4 || G == 8 || (kGroupMma2 && G == 2));
   if (mma_group || (plain && (G == 4 || G == 8) && head_rows * 10 > group_rows * 22)) {
-    // group kernel: splits per KV group over its capacity, G partial slots each
+    // group kernel: splits per KV group over its capacity (then over its
+    // heads' largest global-token count), G partial slots each
     int items = 0;
     p.split_pre[0] = 0;
     p.hslot_pre[0] = 0;
     for (int g = 0; g < c->Hkv; ++g) {
-      const int ns = (c->cap[g] + kGroupChunk - 1) / kGroupChunk;
+      int kmax = 0;
+      for (int j = 0; j < G; ++j) kmax = max(kmax, p.sink[g * G + j]);
+      const int ns = (c->cap[g] + kGroupChunk - 1) / kGroupChunk + (kmax + kGroupChunk - 1) / kGroupChunk;
       p.split_pre[g + 1] = p.split_pre[g] + ns;
       for (int j = 0; j < G; ++j) p.hslot_pre[g * G + j + 1] = p.hslot_pre[g * G + j] + ns;
       items += ns;

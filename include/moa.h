@@ -320,9 +320,10 @@ moa_status moa_workspace_bytes_sink(moa_op op, int32_t B, int32_t Hq, int64_t N,
  * and the global tokens below the band from the global-token rows.
  * sinks: host int32[Hq], 0 <= sinks[h] <= K_{h/(Hq/Hkv)} (else
  * MOA_ERR_CAPACITY).  workspace: moa_workspace_bytes_sink(MOA_OP_DECODE, ...)
- * bytes, zeroed before first use.  One launch: the per-head split-KV kernel,
- * with ceil(k_h / 512) more splits per head over the global-token rows (the
- * group-shared kernels do not take global tokens).  Errors as moa_decode. */
+ * bytes, zeroed before first use.  One launch: the split-KV kernel with more
+ * splits over the global-token rows (per head, or for bf16 d = 128 with 2, 4
+ * or 8 query heads per key/value head per group, the group's rows read once
+ * for all its heads).  Errors as moa_decode. */
 moa_status moa_decode_sink(moa_kv_cache* cache, const void* q, void* o, int32_t Hq,
                            const int32_t* spans, const int32_t* sinks, float scale,
                            void* workspace, size_t ws_bytes, void* stream);

@@ -166,6 +166,8 @@ DECODE_CASES = [
     (2, 16, 2, "bf16", 128, 700, [700, 3, 300, 301, 64, 1, 699, 500,
                                   2, 500, 512, 513, 257, 5, 600, 40], [4] * 16, 2),   # 8 heads per KV head
     (2, 4, 2, "f32", 64, 0, [1, 5, 32, 17], [2, 0, 40, 40], 48),                 # from an empty cache
+    # 4 heads per KV head, global-token counts differing within each group, two global splits
+    (2, 8, 2, "bf16", 128, 2600, [2000, 300, 2500, 64, 1200, 1, 800, 2100], [1500, 0, 3, 1100, 0, 0, 2000, 64], 2),
 ]
 
 
