@@ -665,10 +665,6 @@ constexpr bool kGroupSplitAcc = MOA_GQA_SPLIT_ACC != 0;
 #define MOA_GQA_TILE_FAST 1
 #endif
 constexpr bool kGroupTileFast = MOA_GQA_TILE_FAST != 0;
-#ifndef MOA_GQA_LAZY_RESCALE
-#define MOA_GQA_LAZY_RESCALE 0
-#endif
-constexpr bool kGroupLazyRescale = MOA_GQA_LAZY_RESCALE != 0;
 constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
 constexpr int kMmaWarpRows = kGroupChunk / kDecWarps;  // entries per warp and split
 constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
@@ -948,15 +944,12 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     const float p0 = exp2f(s0 - r0), p1 = exp2f(s1 - r1), p2 = exp2f(s2 - r0), p3 = exp2f(s3 - r1);
     l0 = l0 * cr0 + p0 + p2;
     l1 = l1 * cr1 + p1 + p3;
-    // once the running maxima settle every factor is 1: skip the 32 products
-    if (!kGroupLazyRescale || __any_sync(0xffffffffu, cr0 != 1.f || cr1 != 1.f)) {
 #pragma unroll
-      for (int mb = 0; mb < 8; ++mb) {
-        oacc[mb][0] *= cr0;
-        oacc[mb][1] *= cr1;
-        oacc[mb][2] *= cr0;
-        oacc[mb][3] *= cr1;
-      }
+    for (int mb = 0; mb < 8; ++mb) {
+      oacc[mb][0] *= cr0;
+      oacc[mb][1] *= cr1;
+      oacc[mb][2] *= cr0;
+      oacc[mb][3] *= cr1;
     }
     // P^T into the B-operand layout through the scratch [head][row]
     sPg[h0 * 16 + g4] = __bfloat16_as_ushort(__float2bfloat16_rn(p0));

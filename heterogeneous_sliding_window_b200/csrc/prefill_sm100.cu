@@ -338,8 +338,12 @@ __device__ __forceinline__ float max64(const float* s) {
 // than by MUFU ex2: one in kPolyEvery.  MUFU issues 16 ex2 per clock per SM,
 // which equals the tensor core's pace at d = 128, so moving part of the work
 // to the FMA pipe shortens the softmax, the critical path between two MMAs.
+// Two pairs of every 32 (one in twelve, at pairs 11 and 23) measured best on
+// the current ring layout: 904-908 against 890-893 TFLOP/s for one in eight
+// (25 % density, back to back), 991-1005 against 982-989 at 50 %; one in
+// five or six was slower.
 #ifndef MOA_PREFILL_POLY_EVERY
-#define MOA_PREFILL_POLY_EVERY 8
+#define MOA_PREFILL_POLY_EVERY 12
 #endif
 constexpr int kPolyEvery = MOA_PREFILL_POLY_EVERY;
 
