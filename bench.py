@@ -530,6 +530,7 @@ def run_ours(args):
         cpu_tok, cpu_sample = oracle_decode_sample(args.cpu_seconds)
         cpu_gflops, cpu_p_sample = oracle_prefill_sample(args.cpu_seconds)
         traffic = _ncu_traffic()
+        gqa["traffic"] = traffic.get("gqa")
         result = {
             "metric": METRIC, "value": round(tokens_per_s, 2), "unit": "tokens/s", "n_gpus": ws_n,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -994,7 +995,7 @@ def _ncu_traffic():
     """
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    srcs = {"decode": "decode.cu", "prefill": "prefill_sm100.cu"}
+    srcs = {"decode": "decode.cu", "prefill": "prefill_sm100.cu", "gqa": "decode.cu"}
     out = {}
     try:
         with open(path) as f:
