@@ -642,7 +642,7 @@ def prefill_alone(stream, q, k, v, o, spans, scale, ws, cache, reps=200):
     return ms, clk
 
 
-def chunk_prefill(stream, tf_peak, peak_kind, reps=40):
+def chunk_prefill(stream, tf_peak, peak_kind, reps=150):
     """Chunked prefill into the ring cache: a Vicuna-7B-shaped layer (32 heads,
     d=128, spans at 25 % of 8192) holds the first 4096 tokens of a prompt and
     takes the other 4096 in one moa_prefill_chunk call (window gather,
