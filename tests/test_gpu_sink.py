@@ -299,3 +299,86 @@ def test_bf16_prefill_with_global_tokens_vicuna7b_sampled():
     got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
     assert np.max(np.abs(got - ref)) <= BF16_TOL
     assert cache.positions() == [N]
+
+
+def test_decode_with_global_tokens_llama3_gqa_layer_sampled():
+    """A Llama3-8B-shaped GQA decode layer with global tokens (B=4, 32 query heads on 8 KV heads,
+    d=128, context 8192, 50 % spans, global-token counts from {0, 4, 64, 128, 1024}): the
+    tensor-core group kernel's global splits at full size, sampled (b, h) against the oracle's
+    row decode over the ring and the global rows."""
+    from oracle import rules as orules
+    B, Hq, Hkv, d, N = 4, 32, 8, 128, 8192
+    G = Hq // Hkv
+    a, b = inputs.tables_7b(1001, Hq, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    sinks = inputs.sink_counts(11, Hq)
+    caps, scaps = _group_max(spans, Hkv), _group_max(sinks, Hkv)
+    cache = moa.KVCache(B, Hkv, d, "bf16", caps, sink_capacity=scaps)
+    data = cache.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(31, (data.numel(),)))       # ring rows and global-token rows
+    cache.set_positions([N] * B)
+    host = cache.data_bytes().cpu().numpy().tobytes()
+    scale = 1.0 / math.sqrt(d)
+    qt = inputs.randn_cuda(32, (B, Hq, d))
+    kt = inputs.randn_cuda(33, (B, Hkv, 1, d))
+    vt = inputs.randn_cuda(34, (B, Hkv, 1, d))
+    nb = moa.moa_workspace_bytes_sink(moa.MOA_OP_DECODE, B, Hq, 0, d, spans, sinks)
+    wbuf = torch.zeros(nb + 256, dtype=torch.uint8, device=DEV)
+    ot = _nan((B, Hq, d), torch.bfloat16)
+    moa.moa_decode_append_sink(cache.handle, qt, kt, vt, ot, Hq, spans, sinks, scale,
+                               (wbuf.data_ptr() + 255) // 256 * 256, nb)
+    torch.cuda.synchronize()
+    assert cache.positions() == [N + 1] * B
+    kt64, vt64, qt64, ot64 = (inputs.as_f64(x) for x in (kt, vt, qt, ot))
+    ring_bytes = B * sum(caps) * 2 * d * 2
+    sumK = sum(scaps)
+    rng = np.random.default_rng(12)
+    picks = [(int(rng.integers(B)), int(rng.integers(Hq))) for _ in range(24)] + [(0, 0), (B - 1, Hq - 1)]
+    for bb, hh in picks:
+        g = hh // G
+        K, V = (x.copy() for x in okv.block_from_image(host, bb, g, B, Hkv, d, caps, "bf16"))
+        C = caps[g]
+        K[N % C] = kt64[bb, g, 0]                      # the appended token's slot
+        V[N % C] = vt64[bb, g, 0]
+        Kg = scaps[g]
+        start = (bb * sumK + sum(scaps[:g])) * 2 * d * 2
+        raw = np.frombuffer(host[ring_bytes + start: ring_bytes + start + 2 * Kg * d * 2], dtype="<u2")
+        glob = (raw.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(2, Kg, d)
+        # the band comes through the ring, the global tokens below it from the global-token
+        # rows (the fill is random, so the two copies of a position differ: the call's documented
+        # source decides)
+        t = N + 1
+        keys = oatt.keys_sink(t - 1, spans[hh], sinks[hh])
+        Ks = np.stack([K[p % C] if p >= t - spans[hh] else glob[0][p] for p in keys])
+        Vs = np.stack([V[p % C] if p >= t - spans[hh] else glob[1][p] for p in keys])
+        ref = oatt.attend_row(qt64[bb, hh], Ks, Vs, 0, len(keys) - 1, scale)
+        assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
+
+
+@pytest.mark.parametrize("shape", ["vicuna13b", "llama3_gqa"])
+def test_bf16_prefill_with_global_tokens_full_size_sampled(shape):
+    """Global tokens on the full-size prompts: a Vicuna-13B-shaped layer (40 heads, N=16384, 50 %
+    fixed-local and elastic heads) and the Llama3-8B-shaped GQA prompt (32/8 heads, N=32768, 25 %),
+    global-token counts from {0, 4, 64, 128, 1024}; sampled rows against the oracle."""
+    from oracle import rules as orules
+    d = 128
+    if shape == "vicuna13b":
+        B, Hq, Hkv, N = 1, 40, 40, 16384
+        a, b = inputs.tables_13b_mix(5, Hq, N, 64, 0.5, orules.eval_spans)
+    else:
+        B, Hq, Hkv, N = 1, 32, 8, 32768
+        a, b = inputs.tables_7b(4000, Hq, N, 64, 0.25, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    sinks = inputs.sink_counts(13, Hq)
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn_cuda(41, (B, Hq, N, d))
+    k = inputs.randn_cuda(42, (B, Hkv, N, d))
+    v = inputs.randn_cuda(43, (B, Hkv, N, d))
+    o = _prefill_sink(q, k, v, spans, sinks, scale, "bf16")
+    assert not torch.isnan(o).any()
+    rng = np.random.default_rng(14)
+    rows = [(0, h, i) for h in (0, Hq // 3, Hq - 1) for i in (0, 5, 127, 1100, N // 2, N - 1)]
+    rows += [(0, int(rng.integers(Hq)), int(rng.integers(N))) for _ in range(24)]
+    ref = oatt.prefill_sink(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, sinks, scale, rows=rows)
+    got = np.stack([inputs.as_f64(o[b_, h_, i_]) for b_, h_, i_ in rows])
+    assert np.max(np.abs(got - ref)) <= BF16_TOL
