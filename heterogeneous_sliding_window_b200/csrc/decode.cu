@@ -42,10 +42,6 @@ constexpr int kChunk = MOA_DECODE_CHUNK;   // window entries per split (per-head
 constexpr int kGroupChunk = MOA_GQA_CHUNK;
 static_assert(kGroupChunk >= kChunk, "group split size (the workspace holds the per-head kernel's slots)");
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
-#ifndef MOA_DECODE_PAIRS
-#define MOA_DECODE_PAIRS 0
-#endif
-constexpr bool kDecodePairs = MOA_DECODE_PAIRS != 0;   // packed f32x2 FMAs in the per-head kernel
 #ifndef MOA_GROUP_MMA
 #define MOA_GROUP_MMA 1
 #endif
@@ -236,18 +232,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       float kf[VE];
       Vec16<T>::cvt(kr[u], kf);
       float dot = 0.f;
-      if constexpr (kDecodePairs) {
-        uint64_t d2 = 0;
 #pragma unroll
-        for (int e = 0; e < VE / 2; ++e) d2 = sm100::f2_fma(sm100::f2_pack(qf[2 * e], qf[2 * e + 1]),
-                                                          sm100::f2_pack(kf[2 * e], kf[2 * e + 1]), d2);
-        float d0, d1;
-        sm100::f2_unpack(d2, d0, d1);
-        dot = d0 + d1;
-      } else {
-#pragma unroll
-        for (int e = 0; e < VE; ++e) dot = fmaf(qf[e], kf[e], dot);
-      }
+      for (int e = 0; e < VE; ++e) dot = fmaf(qf[e], kf[e], dot);
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
       sv[u] = (base + u * NG + grp < nrows) ? dot : -INFINITY;
@@ -269,18 +255,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
       l += pu;
       float vf[VE];
       Vec16<T>::cvt(vr[u], vf);
-      if constexpr (kDecodePairs) {
-        const uint64_t p2 = sm100::f2_pack(pu, pu);
 #pragma unroll
-        for (int e = 0; e < VE / 2; ++e) {
-          const uint64_t a2 = sm100::f2_fma(p2, sm100::f2_pack(vf[2 * e], vf[2 * e + 1]),
-                                            sm100::f2_pack(acc[2 * e], acc[2 * e + 1]));
-          sm100::f2_unpack(a2, acc[2 * e], acc[2 * e + 1]);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < VE; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
-      }
+      for (int e = 0; e < VE; ++e) acc[e] = fmaf(pu, vf[e], acc[e]);
     }
   }
 
@@ -643,28 +619,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_kernel(const __grid_
 //     and O^T[128 dims x 8 heads] += V_tile^T . P^T (A = V from ldmatrix.trans).
 // The four warps then merge by log-sum-exp in shared memory and the split's
 // partial (m, l, o) per head is written or, with one split, o itself.
+// A tile whose 16 slots are contiguous and inside the split is copied from one
+// base pointer at constant offsets; others walk the ring row by row.  Splits
+// past a group's window read its global-token rows (each head masks its own
+// count).
 constexpr int kMmaRows = 16;                      // cached rows per tile
 constexpr int kMmaTileBytes = kMmaRows * 128 * 2; // one 16 x 128 bf16 tile
 #ifndef MOA_MMA_STAGES
 #define MOA_MMA_STAGES 2
 #endif
 constexpr int kMmaStages = MOA_MMA_STAGES;        // K/V tiles in flight per warp + 1
-#ifndef MOA_GQA_SPLIT_ACC
-#define MOA_GQA_SPLIT_ACC 0
-#endif
-constexpr bool kGroupSplitAcc = MOA_GQA_SPLIT_ACC != 0;
-// Incremental cp.async addressing in the tensor-core group kernel (1: about
-// 10 fewer instructions per 16-byte copy; 0.164 against 0.167 ms on the
-// layer above).  0 keeps the per-copy address computation.
-#ifndef MOA_GQA_FAST_ADDR
-#define MOA_GQA_FAST_ADDR 1
-#endif
-// ... and the copies of a tile whose 16 slots are contiguous from one base
-// pointer with constant offsets (1), or always the per-copy walk (0).
-#ifndef MOA_GQA_TILE_FAST
-#define MOA_GQA_TILE_FAST 1
-#endif
-constexpr bool kGroupTileFast = MOA_GQA_TILE_FAST != 0;
 constexpr uint32_t kMmaWarpBytes = kMmaStages * 2 * kMmaTileBytes + 256;   // stages + P scratch
 constexpr int kMmaWarpRows = kGroupChunk / kDecWarps;  // entries per warp and split
 constexpr size_t kMmaSmem = (size_t)kDecWarps * kMmaWarpBytes;
@@ -790,7 +754,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   const int ntiles = (wrows + kMmaRows - 1) / kMmaRows;
 
   // issue the copies of tile ti into stage st (rows past the split are zero-filled)
-#if MOA_GQA_FAST_ADDR
   // Lane `lane` copies chunk cc = lane & 15 of tile rows rr0 + 2q, q = 0..7
   // (rr0 = lane >> 4): its slot advances by 2 per row with one wrap test, and
   // its swizzled destinations repeat every four rows (row residues mod 8 are
@@ -808,7 +771,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     // Common case: all 16 rows inside the split, their slots contiguous (no
     // wrap), none the fused append's new entry: one base pointer per lane and
     // constant offsets (two rows, 512 bytes, apart per copy).
-    if (kGroupTileFast && trow + kMmaRows <= nrows && tslot + kMmaRows <= Cw &&
+    if (trow + kMmaRows <= nrows && tslot + kMmaRows <= Cw &&
         !(e_new >= w0 + trow && e_new < w0 + trow + kMmaRows)) {
       const __nv_bfloat16* pk = Kb + (size_t)(tslot + rr0) * D + cc * 8;
 #pragma unroll
@@ -848,45 +811,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
       if (slot >= Cw) slot -= Cw;
     }
   };
-#else
-  auto load_tile = [&](int ti, int st) {
-    const uint32_t dK = sbase + (uint32_t)st * 2 * kMmaTileBytes, dV = dK + kMmaTileBytes;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int i = lane + 32 * q;
-      const int rr = i >> 4, cc = i & 15;
-      const int row = wrow0 + ti * kMmaRows + rr;                // split entry
-      const __nv_bfloat16* srcK = Kb;
-      const __nv_bfloat16* srcV = Vb;
-      uint32_t bytes = 0;
-      if (row < nrows) {
-        bytes = 16;
-        if (w0 + row == e_new) {
-          srcK = kn + cc * 8;
-          srcV = vn + cc * 8;
-          int slot = slot0 + row;
-          if (slot >= Cw) slot -= Cw;
-          // this CTA is the group's only reader of the newest entry: write it to its slot
-          const int4 kx = __ldg(reinterpret_cast<const int4*>(srcK));
-          const int4 vx = __ldg(reinterpret_cast<const int4*>(srcV));
-          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Kb) + (size_t)slot * D + cc * 8) = kx;
-          *reinterpret_cast<int4*>(const_cast<__nv_bfloat16*>(Vb) + (size_t)slot * D + cc * 8) = vx;
-          if (ks_new != nullptr) {
-            *reinterpret_cast<int4*>(ks_new + cc * 8) = kx;
-            *reinterpret_cast<int4*>(ks_new + (size_t)p.scap[g] * D + cc * 8) = vx;
-          }
-        } else {
-          int slot = slot0 + row;
-          if (slot >= Cw) slot -= Cw;
-          srcK = Kb + (size_t)slot * D + cc * 8;
-          srcV = Vb + (size_t)slot * D + cc * 8;
-        }
-      }
-      cp_async16(dK + swz(rr, cc), srcK, bytes);
-      cp_async16(dV + swz(rr, cc), srcV, bytes);
-    }
-  };
-#endif
 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads h0, h1
   float oacc[8][4];
@@ -908,19 +832,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
     cp_async_wait<kMmaStages - 1>();                    // tile ti has landed
     __syncwarp();
     const uint32_t tK = sbase + (uint32_t)(ti % kMmaStages) * 2 * kMmaTileBytes, tV = tK + kMmaTileBytes;
-    // S^T = K . Q^T (two accumulators: two independent MMA chains)
+    // S^T = K . Q^T
     float sacc[4] = {0.f, 0.f, 0.f, 0.f};
     {
-      float sacc2[4] = {0.f, 0.f, 0.f, 0.f};
       const int ar = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         uint32_t a[4];
         ldsm_x4(tK + swz(ar, 2 * kk + (lane >> 4)), a);
-        mma16816((kk & 1) && kGroupSplitAcc ? sacc2 : sacc, a, qb[kk][0], qb[kk][1]);
+        mma16816(sacc, a, qb[kk][0], qb[kk][1]);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[e] += sacc2[e];
     }
     // mask and scale: rows g4 and g4 + 8 of the tile, heads h0 and h1
     const int ra = wrow0 + ti * kMmaRows + g4, rb = ra + 8;
