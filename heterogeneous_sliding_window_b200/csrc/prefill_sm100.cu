@@ -71,13 +71,7 @@ constexpr int kThreads = 384;                    // 3 warpgroups
 // Register split (setmaxnreg): the block launches with 384 x 168 registers;
 // warpgroup 0 (producer, MMA issuer, unit fetcher, cache writer) drops to
 // 120, the two softmax warpgroups rise to 192.
-#ifndef MOA_PREFILL_REGS_CONTROL
-#define MOA_PREFILL_REGS_CONTROL 120
-#endif
-#ifndef MOA_PREFILL_REGS_SOFTMAX
-#define MOA_PREFILL_REGS_SOFTMAX 192
-#endif
-constexpr uint32_t kRegsLaunch = 168, kRegsControl = MOA_PREFILL_REGS_CONTROL, kRegsSoftmax = MOA_PREFILL_REGS_SOFTMAX;
+constexpr uint32_t kRegsLaunch = 168, kRegsControl = 120, kRegsSoftmax = 192;
 static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= kThreads * kRegsLaunch, "register split");
 constexpr int kD = 128;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;   // one 128 x 128 bf16 tile
@@ -950,13 +944,6 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-#ifndef MOA_PREFILL_L2_PROMO
-#define MOA_PREFILL_L2_PROMO 3
-#endif
-// L2 promotion of the tile loads (CUtensorMapL2promotion: 0 none, 1 64 B,
-// 2 128 B, 3 256 B).
-constexpr CUtensorMapL2promotion kL2Promotion = static_cast<CUtensorMapL2promotion>(MOA_PREFILL_L2_PROMO);
-
 bool make_map(CUtensorMap* map, const void* ptr, int32_t N, int64_t heads) {
   auto enc = get_encode();
   if (!enc) return false;
@@ -966,16 +953,13 @@ bool make_map(CUtensorMap* map, const void* ptr, int32_t N, int64_t heads) {
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   kL2Promotion, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 constexpr size_t kOffsOffset = 256;                          // int32 cta_off[kMaxCtas + 1]
 constexpr size_t kUnitsOffset = kOffsOffset + (4 * (kPrefillMaxCtas + 1) + 15) / 16 * 16;
-#ifndef MOA_PREFILL_UNIT_OVERHEAD
-#define MOA_PREFILL_UNIT_OVERHEAD 4
-#endif
-constexpr int64_t kUnitOverheadTiles = MOA_PREFILL_UNIT_OVERHEAD;   // per-unit pipeline fill/drain, in tile steps
+constexpr int64_t kUnitOverheadTiles = 4;     // per-unit pipeline fill/drain, in tile steps
 
 int64_t first_tile_host(int64_t qt, int32_t S) {
   return std::max<int64_t>(0, qt * kTileM - S + 1) / kTileN;
