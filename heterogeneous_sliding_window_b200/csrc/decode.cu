@@ -50,10 +50,6 @@ constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads 
 #define MOA_DECODE_BATCH_FAST 1
 #endif
 constexpr bool kDecodeBatchFast = MOA_DECODE_BATCH_FAST != 0;   // contiguous batches from one base pointer
-#ifndef MOA_DECODE_MIN_BLOCKS
-#define MOA_DECODE_MIN_BLOCKS 1
-#endif
-constexpr int kDecodeMinBlocks = MOA_DECODE_MIN_BLOCKS;   // resident CTAs per SM asked of the register allocator
 #ifndef MOA_GROUP_MMA
 #define MOA_GROUP_MMA 1
 #endif
@@ -132,7 +128,7 @@ __device__ __forceinline__ void step_counted(const DecodeParams& p, int b, int64
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kDecThreads, kDecodeMinBlocks) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int VE = Vec16<T>::N;     // elements per 16-byte vector
   constexpr int LPR = D / VE;         // lanes per cached row
   constexpr int RPW = 32 / LPR;       // row groups per warp
