@@ -975,14 +975,18 @@ def global_tokens(stream, peaks, read_gbs, reps_prefill=100, reps_decode=300):
     ms, clk = back_to_back(stream, lambda: moa.moa_decode_append_sink(c.handle, dq, dk, dv, do, D_H, dsp, sinks, scale,
                                                                       wptr, nb, stream), reps_decode)
     c.positions()
-    layer_bytes = D_B * sum(2 * (S + kk) * D_D * 2 for S, kk in zip(dsp, sinks)) + 6 * D_B * D_H * D_D * 2
+    # each head reads its band and the global tokens below it: min(k_h, t - S_h) rows at context t
+    layer_bytes = (D_B * sum(2 * (S + min(kk, D_N - S)) * D_D * 2 for S, kk in zip(dsp, sinks))
+                   + 6 * D_B * D_H * D_D * 2)
     gbs = layer_bytes / (ms * 1e-3) / 1e9
     out["decode"] = {"workload": "vicuna7b-shaped decode layer B=32 H=32 d=128 ctx 4096 density 0.50 + global "
                                  "tokens, fused append", "ms": round(ms, 4), "bytes_per_launch": int(layer_bytes),
                      "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
                      "frac_of_read_only": round(gbs / read_gbs, 4),
                      "tokens_per_s_one_layer": round(D_B / (ms * 1e-3), 1),
-                     "kernel": "decode_kernel<bf16,128> with global-token splits", "clocks": clk}
+                     "kernel": "decode_kernel<bf16,128> with global-token splits", "clocks": clk,
+                     "note": "back to back on one layer's cache; the global-token rows, re-read by every call, "
+                             "partly come from L2"}
     del c, wbuf
     torch.cuda.empty_cache()
     return out
