@@ -334,16 +334,16 @@ __device__ __forceinline__ float max64(const float* s) {
   return max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
-// Pairs of exponentials taken by the cubic on the FMA pipe (exp2_poly2) rather
-// than by MUFU ex2: one in kPolyEvery.  MUFU issues 16 ex2 per clock per SM,
-// which equals the tensor core's pace at d = 128, so moving part of the work
-// to the FMA pipe shortens the softmax, the critical path between two MMAs.
-// Two pairs of every 32 (one in twelve, at pairs 11 and 23) measured best on
-// the current ring layout: 904-908 against 890-893 TFLOP/s for one in eight
-// (25 % density, back to back), 991-1005 against 982-989 at 50 %; one in
-// five or six was slower.
+// Pairs of exponentials that may be taken by the cubic on the FMA pipe
+// (exp2_poly2) rather than by MUFU ex2: one in kPolyEvery, none when 0.
+// MUFU issues 16 ex2 per clock per SM, the tensor core's pace at d = 128, and
+// with three Q slots and two-stage rings one pair in eight on the cubic paid.
+// With two Q slots, a three-stage K ring and tile B's first S in the prologue
+// the fewer the better: none measured 936 TFLOP/s against 922 for one pair in
+// 32, 909 for two in 32 and 890 for four (25 % density, back to back), and
+// 1004-1035 against 988-1000 for two in 32 at 50 %.
 #ifndef MOA_PREFILL_POLY_EVERY
-#define MOA_PREFILL_POLY_EVERY 12
+#define MOA_PREFILL_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = MOA_PREFILL_POLY_EVERY;
 
@@ -355,7 +355,7 @@ __device__ __forceinline__ float exp_half(const float* s, float c, float neg, ui
   for (int j = 0; j < 32; ++j) {
     const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, n2);
     uint64_t p2;
-    if (j % kPolyEvery == kPolyEvery - 1) {
+    if (kPolyEvery > 0 && j % kPolyEvery == kPolyEvery - 1) {
       p2 = exp2_poly2(x2);
     } else {
       float x0, x1;
