@@ -346,6 +346,7 @@ __device__ __forceinline__ float max64(const float* s) {
 #define MOA_PREFILL_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = MOA_PREFILL_POLY_EVERY;
+constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;   // the modulus of the test below, never 0
 
 // p = 2^(s * c - m) for 64 scores as bf16 pairs w[32]; returns the fp32 sum.
 __device__ __forceinline__ float exp_half(const float* s, float c, float neg, uint32_t* w) {
@@ -355,7 +356,7 @@ __device__ __forceinline__ float exp_half(const float* s, float c, float neg, ui
   for (int j = 0; j < 32; ++j) {
     const uint64_t x2 = f2_fma(f2_pack(s[2 * j], s[2 * j + 1]), c2, n2);
     uint64_t p2;
-    if (kPolyEvery > 0 && j % kPolyEvery == kPolyEvery - 1) {
+    if (kPolyEvery > 0 && j % kPolyMod == kPolyMod - 1) {
       p2 = exp2_poly2(x2);
     } else {
       float x0, x1;
