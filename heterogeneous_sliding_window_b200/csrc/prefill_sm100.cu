@@ -152,6 +152,7 @@ struct PrefillParams {
   const int64_t* t;
   int32_t Hq, Hkv, G;
   int32_t stall;                 // self-test of the bounded waits: the fetcher publishes nothing
+  int32_t o_wide;                // o is 32-byte aligned: output rows go out in 32-byte stores
   float scale_log2;
   int32_t span[MOA_MAX_HEADS];
   int32_t sink[MOA_MAX_HEADS];   // global tokens per head (keys j < sink[h] are kept too), 0: none
@@ -374,6 +375,44 @@ __device__ __forceinline__ float exp_half(const float* s, float c, float neg, ui
   return a + b;
 }
 
+// Output rows of one finished query tile (its uc-th): O / l -> bf16 (round to
+// nearest even) -> global.  The O buffer is released as soon as it is in
+// registers, so the next unit's PVs of this tile stream can start while the
+// stores go out.  False when the wait for O gave up.
+__device__ __forceinline__ bool write_o(const PrefillParams& p, const Ctx& c, uint32_t tO, int X, uint32_t uc,
+                                        int zq, int i_row, float l_run) {
+  if (!c.wait_warp(B_OFULL0 + X, uc & 1)) return false;
+  tc_fence_after();
+  const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+  uint32_t pk[64];
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t rr[32];
+    tmem_ld32(tO + cc * 32, rr);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      pk[16 * cc + j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * inv, __uint_as_float(rr[2 * j + 1]) * inv);
+  }
+  tc_fence_before();
+  c.arrive_warp(B_OEMPTY0 + X);
+  const int o_row = i_row - p.q_off;
+  if (o_row < p.Nq) {
+    // Each thread writes its own 256-byte row, so one store instruction
+    // touches 32 rows; 32-byte stores halve the instructions and write whole
+    // sectors.
+    __nv_bfloat16* orow_p = reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)zq * p.Nq + (size_t)o_row) * kD;
+    if (p.o_wide) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) st_global_v8(orow_p + 16 * j, pk + 8 * j);
+    } else {
+      uint4* orow = reinterpret_cast<uint4*>(orow_p);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) orow[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    }
+  }
+  return true;
+}
+
 __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& c, uint32_t tmem,
                                              int X, int warp, int lane) {
   const int quarter = warp & 3;                      // TMEM lane quarter this warp may access
@@ -453,31 +492,7 @@ __device__ __forceinline__ void softmax_role(const PrefillParams& p, const Ctx& 
       tc_fence_before();
       c.arrive_warp(B_PFULL0 + X);
     }
-    // Output rows: O / l -> bf16 (round to nearest even) -> global.  The O
-    // buffer is released as soon as it is in registers, so the next unit's
-    // PVs of this tile stream can start while the stores go out.
-    if (!c.wait_warp(B_OFULL0 + X, uc & 1)) return;
-    tc_fence_after();
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    uint32_t pk[64];
-#pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      uint32_t rr[32];
-      tmem_ld32(tO + cc * 32, rr);
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        pk[16 * cc + j] = pack_bf16x2(__uint_as_float(rr[2 * j]) * inv, __uint_as_float(rr[2 * j + 1]) * inv);
-    }
-    tc_fence_before();
-    c.arrive_warp(B_OEMPTY0 + X);
-    const int o_row = i_row - p.q_off;
-    if (o_row < p.Nq) {
-      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                             ((size_t)x.zq * p.Nq + (size_t)o_row) * kD);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) orow[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-    }
-    ++uc;
+    if (!write_o(p, c, tO, X, uc++, x.zq, i_row, l_run)) return;
   }
 }
 
@@ -1163,6 +1178,7 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   p.cta_off = reinterpret_cast<const int32_t*>((char*)ws + kOffsOffset);
   p.units = reinterpret_cast<const int4*>((char*)ws + kUnitsOffset);
   p.o = o;
+  p.o_wide = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
   p.N = Nk;
   p.Nq = Nq;
   p.q_off = q_off;

@@ -108,6 +108,31 @@ def test_bf16_prefill_matches_oracle(case):
     assert err <= BF16_TOL, err
 
 
+def test_bf16_prefill_output_only_16_byte_aligned():
+    """Output rows go out in 32-byte stores when o is 32-byte aligned, else in
+    16-byte stores: an o 16 bytes past a 32-byte boundary takes the second path,
+    and nothing outside o is written."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 700, 128
+    spans = [1, 129, 300, 700]
+    scale = 1.0 / math.sqrt(d)
+    q = inputs.randn(21, (B, Hq, N, d))
+    k = inputs.randn(22, (B, Hkv, N, d))
+    v = inputs.randn(23, (B, Hkv, N, d))
+    n = B * Hq * N * d
+    flat = _nan_like((n + 32,), torch.bfloat16)
+    off = ((16 - flat.data_ptr() % 32) % 32) // 2
+    o = flat[off:off + n].view(B, Hq, N, d)
+    assert o.data_ptr() % 32 == 16
+    ws = moa.Workspace(moa.MOA_OP_PREFILL, B, Hq, N, d, spans)
+    moa.moa_prefill(q.to(DEV), k.to(DEV), v.to(DEV), o, B, Hq, Hkv, N, d, "bf16", spans, scale, ws.ptr, ws.nbytes)
+    moa.moa_workspace_check(ws.ptr)
+    torch.cuda.synchronize()
+    ref = oatt.prefill(inputs.as_f64(q), inputs.as_f64(k), inputs.as_f64(v), spans, scale)
+    err = np.max(np.abs(inputs.as_f64(o) - ref))
+    assert err <= BF16_TOL, err
+    assert torch.isnan(flat[:off]).all() and torch.isnan(flat[off + n:]).all()
+
+
 def test_bf16_prefill_scores_growing_along_the_sequence():
     """Key norms grow with position, so later tiles' maxima jump far above the
     running maximum (the kernel's rescale path) and early tiles underflow."""
