@@ -58,6 +58,7 @@ extern "C" const char* moa_status_string(moa_status s) {
     case MOA_ERR_UNSUPPORTED: return "MOA_ERR_UNSUPPORTED";
     case MOA_ERR_CUDA: return "MOA_ERR_CUDA";
     case MOA_ERR_TIMEOUT: return "MOA_ERR_TIMEOUT";
+    case MOA_ERR_HOST: return "MOA_ERR_HOST";
   }
   return "MOA_ERR_UNKNOWN";
 }
@@ -236,7 +237,7 @@ extern "C" moa_status moa_prefill_stall_test(const void* q, const void* k, const
   if (!q || !k || !v || !o) return MOA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return MOA_ERR_INVALID_ARG;
   if (!ws || ((uintptr_t)ws & 255u) != 0 || ws_bytes < prefill_workspace_bytes(1, 1, 128)) return MOA_ERR_WORKSPACE;
-  return launch_prefill_stall_test(q, k, v, o, ws, ws_bytes, (cudaStream_t)stream);
+  return guarded([&] { return launch_prefill_stall_test(q, k, v, o, ws, ws_bytes, (cudaStream_t)stream); });
 }
 
 extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, const int32_t* spans,
@@ -247,11 +248,13 @@ extern "C" moa_status moa_prefill_schedule(int32_t B, int32_t Hq, int64_t N, con
     return MOA_ERR_INVALID_ARG;
   for (int32_t h = 0; h < Hq; ++h)
     if (spans[h] < 1) return MOA_ERR_INVALID_ARG;
-  const std::vector<int32_t> rows = prefill_schedule_rows(B, Hq, (int32_t)N, spans, n_ctas);
-  const int64_t n = (int64_t)rows.size() / 7;
-  std::copy(rows.begin(), rows.begin() + 7 * std::min(n, cap), rows_out);
-  *n_rows_out = n;
-  return MOA_OK;
+  return guarded([&] {
+    const std::vector<int32_t> rows = prefill_schedule_rows(B, Hq, (int32_t)N, spans, n_ctas);
+    const int64_t n = (int64_t)rows.size() / 7;
+    std::copy(rows.begin(), rows.begin() + 7 * std::min(n, cap), rows_out);
+    *n_rows_out = n;
+    return MOA_OK;
+  });
 }
 
 static moa_status prefill_common(const void* q, const void* k, const void* v, void* o, int32_t B,
@@ -263,7 +266,9 @@ extern "C" moa_status moa_prefill(const void* q, const void* k, const void* v, v
                                   int32_t Hq, int32_t Hkv, int64_t N, int32_t d, moa_dtype dtype,
                                   const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                   moa_kv_cache* fill, void* stream) {
-  return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, nullptr, scale, ws, ws_bytes, fill, stream);
+  return guarded([&] {
+    return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, nullptr, scale, ws, ws_bytes, fill, stream);
+  });
 }
 
 extern "C" moa_status moa_prefill_sink(const void* q, const void* k, const void* v, void* o, int32_t B,
@@ -271,7 +276,9 @@ extern "C" moa_status moa_prefill_sink(const void* q, const void* k, const void*
                                        const int32_t* spans, const int32_t* sinks, float scale, void* ws,
                                        size_t ws_bytes, moa_kv_cache* fill, void* stream) {
   if (!sinks) return MOA_ERR_INVALID_ARG;
-  return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, sinks, scale, ws, ws_bytes, fill, stream);
+  return guarded([&] {
+    return prefill_common(q, k, v, o, B, Hq, Hkv, N, d, dtype, spans, sinks, scale, ws, ws_bytes, fill, stream);
+  });
 }
 
 static moa_status prefill_common(const void* q, const void* k, const void* v, void* o, int32_t B,
@@ -358,7 +365,9 @@ extern "C" moa_status moa_prefill_chunk(moa_kv_cache* c, const void* q, const vo
   if (st != MOA_OK) return st;
   if (!ws || ((uintptr_t)ws & 255u) != 0) return MOA_ERR_WORKSPACE;
   if (ws_bytes < prefill_chunk_workspace_bytes(c->B, Hq, c->Hkv, n, spans)) return MOA_ERR_WORKSPACE;
-  return launch_prefill_chunk(c, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
+  return guarded([&] {
+    return launch_prefill_chunk(c, q, k, v, o, Hq, n, spans, scale, ws, ws_bytes, (cudaStream_t)stream);
+  });
 }
 
 // Shared checks and dispatch of the decode entry points (k, v: the fused
@@ -394,25 +403,25 @@ extern "C" moa_status moa_decode_append(moa_kv_cache* c, const void* q, const vo
                                         void* o, int32_t Hq, const int32_t* spans, float scale, void* ws,
                                         size_t ws_bytes, void* stream) {
   if (!k || !v) return MOA_ERR_INVALID_ARG;
-  return decode_common(c, q, k, v, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream);
+  return guarded([&] { return decode_common(c, q, k, v, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream); });
 }
 
 extern "C" moa_status moa_decode_append_sink(moa_kv_cache* c, const void* q, const void* k, const void* v,
                                              void* o, int32_t Hq, const int32_t* spans, const int32_t* sinks,
                                              float scale, void* ws, size_t ws_bytes, void* stream) {
   if (!k || !v || !sinks) return MOA_ERR_INVALID_ARG;
-  return decode_common(c, q, k, v, o, Hq, spans, sinks, scale, ws, ws_bytes, stream);
+  return guarded([&] { return decode_common(c, q, k, v, o, Hq, spans, sinks, scale, ws, ws_bytes, stream); });
 }
 
 extern "C" moa_status moa_decode_sink(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                                       const int32_t* spans, const int32_t* sinks, float scale, void* ws,
                                       size_t ws_bytes, void* stream) {
   if (!sinks) return MOA_ERR_INVALID_ARG;
-  return decode_common(c, q, nullptr, nullptr, o, Hq, spans, sinks, scale, ws, ws_bytes, stream);
+  return guarded([&] { return decode_common(c, q, nullptr, nullptr, o, Hq, spans, sinks, scale, ws, ws_bytes, stream); });
 }
 
 extern "C" moa_status moa_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq,
                                  const int32_t* spans, float scale, void* ws, size_t ws_bytes,
                                  void* stream) {
-  return decode_common(c, q, nullptr, nullptr, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream);
+  return guarded([&] { return decode_common(c, q, nullptr, nullptr, o, Hq, spans, nullptr, scale, ws, ws_bytes, stream); });
 }

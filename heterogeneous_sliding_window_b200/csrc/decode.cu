@@ -40,6 +40,9 @@ constexpr int kChunk = MOA_DECODE_CHUNK;   // window entries per split (per-head
 #define MOA_GQA_CHUNK 1024
 #endif
 constexpr int kGroupChunk = MOA_GQA_CHUNK;
+// Number of splits of x entries, chunk at a time (64-bit, so spans up to
+// INT32_MAX do not wrap).
+__host__ __device__ inline int splits_of(int x, int chunk) { return (int)(((long long)x + chunk - 1) / chunk); }
 static_assert(kGroupChunk >= kChunk, "group split size (the workspace holds the per-head kernel's slots)");
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
 // Batches whose rows are contiguous in the ring load from one base pointer at
@@ -162,7 +165,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int Seff = (int)(tb < (int64_t)p.span[h] ? tb : (int64_t)p.span[h]);
-  const int nwin = (p.span[h] + kChunk - 1) / kChunk;  // window splits of head h
+  const int nwin = splits_of(p.span[h], kChunk);       // window splits of head h
   // Splits s >= nwin read the global tokens below the window: positions
   // 0 .. min(k_h, tb - Seff) - 1, at rows of the same index.
   const bool gsplit = s >= nwin;
@@ -712,7 +715,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_group_mma_kernel(const __g
   // Splits s >= nwin cover the group's global tokens below its heads' windows:
   // positions 0 .. GW - 1 (the union over the group's heads), rows of the
   // global-token region, which do not wrap.
-  const int nwin = (C + kGroupChunk - 1) / kGroupChunk;
+  const int nwin = splits_of(C, kGroupChunk);
   const bool gsplit = s >= nwin;
   int GW = 0;
   if (gsplit) {
@@ -1045,15 +1048,15 @@ DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* span
   DecodeLayout L;
   int items = 0, max_s = 0, max_k = 0;
   for (int h = 0; h < Hq; ++h) {
-    items += (spans[h] + kChunk - 1) / kChunk;
+    items += splits_of(spans[h], kChunk);
     max_s = max_s > spans[h] ? max_s : spans[h];
     if (sinks) {
-      items += (sinks[h] + kChunk - 1) / kChunk;   // global-token splits
+      items += splits_of(sinks[h], kChunk);   // global-token splits
       max_k = max_k > sinks[h] ? max_k : sinks[h];
     }
   }
   L.items_per_b = items;
-  const size_t slots = (size_t)Hq * ((max_s + kChunk - 1) / kChunk + (max_k + kChunk - 1) / kChunk);
+  const size_t slots = (size_t)Hq * ((size_t)splits_of(max_s, kChunk) + (size_t)splits_of(max_k, kChunk));
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   L.ctr_off = 256;
   L.bctr_off = L.ctr_off + up((size_t)B * Hq * 4);
@@ -1096,7 +1099,7 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   for (int h = 0; h < Hq; ++h) {
     p.span[h] = spans[h];
     p.sink[h] = sinks ? sinks[h] : 0;
-    p.split_pre[h + 1] = p.split_pre[h] + (spans[h] + kChunk - 1) / kChunk + (p.sink[h] + kChunk - 1) / kChunk;
+    p.split_pre[h + 1] = p.split_pre[h] + splits_of(spans[h], kChunk) + splits_of(p.sink[h], kChunk);
   }
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
@@ -1136,7 +1139,7 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
     for (int g = 0; g < c->Hkv; ++g) {
       int kmax = 0;
       for (int j = 0; j < G; ++j) kmax = max(kmax, p.sink[g * G + j]);
-      const int ns = (c->cap[g] + kGroupChunk - 1) / kGroupChunk + (kmax + kGroupChunk - 1) / kGroupChunk;
+      const int ns = splits_of(c->cap[g], kGroupChunk) + splits_of(kmax, kGroupChunk);
       p.split_pre[g + 1] = p.split_pre[g] + ns;
       for (int j = 0; j < G; ++j) p.hslot_pre[g * G + j + 1] = p.hslot_pre[g * G + j] + ns;
       items += ns;

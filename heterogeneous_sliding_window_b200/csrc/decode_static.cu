@@ -68,7 +68,7 @@ extern "C" moa_status moa_decode_static_ws(moa_kv_cache* c, const void* q, void*
   const size_t need = moa::decode_workspace_bytes(c->B, Hq, c->d, spans);
   if (need > kStaticScratchBytes) return MOA_ERR_WORKSPACE;
   void* scratch = nullptr;
-  moa_status st = scratch_for_current_device(&scratch);
+  moa_status st = moa::guarded([&] { return scratch_for_current_device(&scratch); });
   if (st != MOA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   // The header and the per-(b, h) tickets must start at zero; the partials
@@ -76,5 +76,5 @@ extern "C" moa_status moa_decode_static_ws(moa_kv_cache* c, const void* q, void*
   const size_t zero_bytes = 256 + (size_t)c->B * Hq * sizeof(uint32_t);
   const cudaError_t e = cudaMemsetAsync(scratch, 0, zero_bytes, s);
   if (e != cudaSuccess) return moa::cuda_fail(e, "static scratch memset");
-  return moa::launch_decode(c, q, o, Hq, spans, scale, scratch, kStaticScratchBytes, s);
+  return moa::guarded([&] { return moa::launch_decode(c, q, o, Hq, spans, scale, scratch, kStaticScratchBytes, s); });
 }

@@ -53,6 +53,18 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* do
 // variable MOA_VERBOSE is set (the status alone cannot carry the reason);
 // clears the runtime's pending error.
 moa_status cuda_fail(cudaError_t e, const char* where);
+// Runs an entry point's host-side work.  A C++ exception (a schedule's
+// vectors that cannot be allocated, a lock that cannot be taken) becomes
+// MOA_ERR_HOST instead of crossing the C boundary; the throwing paths run
+// before any launch.
+template <class F>
+moa_status guarded(F&& f) noexcept {
+  try {
+    return f();
+  } catch (...) {
+    return MOA_ERR_HOST;
+  }
+}
 inline moa_status check_launch(const char* where) {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? MOA_OK : cuda_fail(e, where);

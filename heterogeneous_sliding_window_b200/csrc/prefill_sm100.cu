@@ -274,7 +274,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const PrefillParams& p, const in
   x.hasB = (long long)x.m[1] * 128 < (long long)p.N;
   x.lo[1] = max(first_key_tile(x.m[1], x.S), kmin >> 7);
   x.R = x.hasB ? x.m[1] : x.m[0];
-  x.ks = (x.k + 127) >> 7;
+  x.ks = (int)(((long long)x.k + 127) >> 7);
   x.P = min(x.ks, x.hasB ? x.lo[1] : x.lo[0]);
   x.Lb = max(x.lo[0], x.P);
   x.first[0] = x.ks > 0 ? 0 : x.lo[0];
@@ -989,7 +989,7 @@ int64_t first_tile_host(int64_t qt, int32_t S) {
 // is its (query tile, key tile) pairs plus a fixed per-unit overhead.
 PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t* spans, int32_t n_ctas,
                                  int32_t m0, const int32_t* sinks) {
-  const int64_t M = (N + kTileM - 1) / kTileM;      // key tiles; query tiles are m0 .. M-1
+  const int64_t M = ((int64_t)N + kTileM - 1) / kTileM;   // key tiles; query tiles are m0 .. M-1
   const int64_t per_head = std::max<int64_t>(0, (M - m0 + 1) / 2);
   const int64_t n_units = (int64_t)B * Hq * per_head;
   // unit u = (b * Hq + h) * per_head + k covers query tiles m0 + 2k and m0 + 2k + 1
@@ -1069,7 +1069,7 @@ PrefillSchedule prefill_schedule(int32_t B, int32_t Hq, int32_t N, const int32_t
 // query tile, in the order each CTA takes its units.
 std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, const int32_t* spans,
                                            int32_t n_ctas) {
-  const int64_t M = (N + kTileM - 1) / kTileM;
+  const int64_t M = ((int64_t)N + kTileM - 1) / kTileM;
   const PrefillSchedule sch = prefill_schedule(B, Hq, N, spans, n_ctas);
   std::vector<int32_t> rows;
   rows.reserve((size_t)B * Hq * M * 7);
@@ -1085,7 +1085,7 @@ std::vector<int32_t> prefill_schedule_rows(int32_t B, int32_t Hq, int32_t N, con
 }
 
 size_t prefill_workspace_bytes(int32_t B, int32_t Hq, int64_t N) {
-  const int64_t M = (N + kTileM - 1) / kTileM;
+  const int64_t M = ((int64_t)N + kTileM - 1) / kTileM;
   return kUnitsOffset + (size_t)B * Hq * M * 16;
 }
 
@@ -1167,7 +1167,7 @@ moa_status launch_prefill_bf16_rows(const void* q, const void* k, const void* v,
   // uploaded in one copy.  The pageable source is staged by the runtime
   // before cudaMemcpyAsync returns.
   const int32_t m0 = q_off / kTileM;
-  const int64_t Mq = (Nq + kTileM - 1) / kTileM;
+  const int64_t Mq = ((int64_t)Nq + kTileM - 1) / kTileM;
   const int64_t n_units = (int64_t)B * Hq * ((Mq + 1) / 2);
   const int32_t grid = (int32_t)std::min<int64_t>({n_units, (int64_t)sm_count(), (int64_t)kPrefillMaxCtas});
   const std::shared_ptr<const UnitBlob> sch = unit_blob(B, Hq, Nk, spans, grid, m0, sinks);

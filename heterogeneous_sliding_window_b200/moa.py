@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoa.so")
 
 MOA_OK, MOA_ERR_INVALID_ARG, MOA_ERR_CAPACITY, MOA_ERR_WORKSPACE = 0, 1, 2, 3
-MOA_ERR_UNSUPPORTED, MOA_ERR_CUDA, MOA_ERR_TIMEOUT = 4, 5, 6
+MOA_ERR_UNSUPPORTED, MOA_ERR_CUDA, MOA_ERR_TIMEOUT, MOA_ERR_HOST = 4, 5, 6, 7
 MOA_F32, MOA_BF16 = 0, 1
 MOA_OP_PREFILL, MOA_OP_DECODE = 0, 1
 

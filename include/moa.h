@@ -19,7 +19,10 @@
  *    Device work is enqueued asynchronously on it; the caller keeps every
  *    buffer alive until that work has completed.
  *  - Argument errors are detected on the host, return a status and launch
- *    nothing.  Launch failures return MOA_ERR_CUDA.  Nothing calls exit/abort.
+ *    nothing.  Launch failures return MOA_ERR_CUDA.  Host memory that a
+ *    launch's plan needs (the prefill's work schedule) and cannot get returns
+ *    MOA_ERR_HOST, with nothing launched.  Nothing calls exit/abort, and no
+ *    C++ exception leaves the library.
  *  - Tensors are dense, row-major, 16-byte aligned:
  *      q, o : [B, Hq,  N, d]     k, v : [B, Hkv, N, d]     (prefill)
  *      q, o : [B, Hq,  d]        k, v : [B, Hkv, n_tok, d] (decode / append)
@@ -45,7 +48,8 @@ typedef enum {
   MOA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than moa_workspace_bytes */
   MOA_ERR_UNSUPPORTED = 4,  /* valid request the library does not implement (e.g. bf16 d=64) */
   MOA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
-  MOA_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (error word set) */
+  MOA_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up (error word set) */
+  MOA_ERR_HOST = 7          /* host-side memory for a launch's plan could not be had (nothing launched) */
 } moa_status;
 
 typedef enum { MOA_F32 = 0, MOA_BF16 = 1 } moa_dtype;

@@ -185,6 +185,17 @@ def test_prefill_schedule_arguments():
         moa.moa_prefill_schedule(1, 1, 128, [64], 1025)
 
 
+def test_host_memory_failure_is_a_status():
+    """A plan whose host vectors cannot be allocated (about 2^61 work units) comes back as
+    MOA_ERR_HOST: no C++ exception crosses the C boundary, and the process goes on."""
+    with pytest.raises(moa.MoaError) as e:
+        moa.moa_prefill_schedule(2**31 - 1, 128, 2**31 - 1, [1] * 128, 148)
+    assert e.value.status == moa.MOA_ERR_HOST
+    lib = moa.load()
+    assert lib.moa_status_string(moa.MOA_ERR_HOST) == b"MOA_ERR_HOST"
+    assert len(moa.moa_prefill_schedule(1, 1, 128, [64], 1)) == 1
+
+
 def test_kv_sizes_match_layout():
     for B, Hkv, d, caps, dt, eb in [(2, 2, 4 * 16, [2, 3], "bf16", 2), (31, 3, 128, [5, 1, 9], "f32", 4),
                                    (32, 32, 128, [2048] * 32, "bf16", 2)]:
