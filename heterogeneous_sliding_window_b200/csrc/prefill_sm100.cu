@@ -550,7 +550,7 @@ __device__ __forceinline__ void mma_role(const PrefillParams& p, const Ctx& c, u
   const uint32_t tSA = tmem + kColS, tSB = tmem + kColS + 128u;
   const uint32_t tOA = tmem + kColO, tOB = tmem + kColO + 128u;
   uint32_t kst = 0, kph = 0, vst = 0, vph = 0;       // K and V ring positions
-  uint32_t nq = 0;                                   // Q tiles used so far (slot nq % 3)
+  uint32_t nq = 0;                                   // Q tiles used so far (slot nq % kQSlots)
   uint32_t tpA = 0, tpB = 0, ucA = 0, ucB = 0;       // PV tiles and units per stream
   uint32_t ui = 0;                                   // unit records read
   int4 U;
