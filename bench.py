@@ -514,6 +514,7 @@ def run_ours(args):
     d2h = sum(x.numel() * x.element_size() for x in h_o)
     gqa = gqa_decode_layer(stream)
     chunk = chunk_prefill(stream, tf_peak, peak_kind)
+    dgraph = decode_graph_b1(stream)
     p_alone_ms, p_alone_clk = prefill_alone(stream, q, k, v, o, p_spans, p_scale, p_ws, p_cache)
     p_alone_tf = p_flops / (p_alone_ms * 1e-3) / 1e12
     read_gbs = read_only_gbs([c.data_bytes() for c in caches[:4]], stream)
@@ -571,6 +572,7 @@ def run_ours(args):
                     "note": "decode step through the C ABI from pinned host q/k/v to host o; copies on a "
                             "second stream overlap the kernels"},
             "gqa_decode": gqa,
+            "decode_graph_b1": dgraph,
             "prefill_chunk": chunk,
             "vicuna13b": v13,
             "llama3_gqa_prefill": l3,
@@ -753,6 +755,73 @@ def gqa_decode_layer(stream, reps=300):
             "ms": round(ms, 4), "group_window_bytes": group_bytes, "per_head_window_bytes": head_bytes,
             "gbs_of_group_bytes": round(group_bytes / (ms * 1e-3) / 1e9, 1),
             "tokens_per_s_one_layer": round(B / (ms * 1e-3), 1), "clocks": clk}
+
+
+def decode_graph_b1(stream, reps=100):
+    """Batch-1 decode step of the Vicuna-7B layout (32 layers x 32 heads, d=128, context 4096,
+    50 % density): 32 fused append+attend launches per step, issued one by one from the host,
+    against the same step captured once in a CUDA graph and replayed.  At batch 1 each launch
+    reads about 33 MB, so per-launch host work is a visible share of the step."""
+    import torch
+    from heterogeneous_sliding_window_b200 import inputs, moa
+    B, H, d, L, ctx = 1, D_H, D_D, D_L, D_N
+    scale = 1.0 / math.sqrt(d)
+    layers = []
+    for layer in range(L):
+        a, b = inputs.tables_7b(D_SEED + layer, H, ctx, BLOCK, D_DENSITY, moa.moa_rules_eval)
+        sp = moa.moa_rules_eval(a, b, ctx, BLOCK)
+        c = moa.KVCache(B, H, d, "bf16", sp)
+        data = c.data_bytes().view(torch.bfloat16)
+        data.copy_(inputs.randn_cuda(3000 + layer, (data.numel(),)))
+        c.set_positions([ctx])
+        ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, sp)
+        bufs = (inputs.randn_cuda(3100 + layer, (B, H, d)), inputs.randn_cuda(3200 + layer, (B, H, 1, d)),
+                inputs.randn_cuda(3300 + layer, (B, H, 1, d)), torch.empty((B, H, d), dtype=torch.bfloat16,
+                                                                           device="cuda"))
+        layers.append((sp, c, ws, bufs))
+    step_bytes = sum(B * sum(2 * S * d * 2 for S in sp) + 6 * B * H * d * 2 for sp, _, _, _ in layers)
+
+    def step(s):
+        for sp, c, ws, (q, k, v, o) in layers:
+            moa.moa_decode_append(c.handle, q, k, v, o, H, sp, scale, ws.ptr, ws.nbytes, s)
+
+    def timed(run):
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        clocks = ClockSampler.for_current_device()
+        clocks.start()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps, clocks.stop()
+
+    eager_ms, eager_clk = timed(lambda: step(stream))
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(side)                                  # first use outside the capture
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=side):
+        step(side)
+    graph_ms, graph_clk = timed(graph.replay)
+    torch.cuda.synchronize()
+    del graph
+    for _, c, _, _ in layers:
+        c.positions()
+        c.close()
+    return {"workload": "vicuna7b-shaped decode step at batch 1: 32 layers x 32 heads, d=128, ctx 4096, "
+                        "density 0.50, append and attend fused per layer",
+            "launches_per_step": L, "bytes_per_step": step_bytes,
+            "eager": {"us_per_step": round(eager_ms * 1e3, 1), "tokens_per_s": round(B / (eager_ms * 1e-3), 1),
+                      "gbs": round(step_bytes / (eager_ms * 1e-3) / 1e9, 1), "clocks": eager_clk},
+            "graph": {"us_per_step": round(graph_ms * 1e3, 1), "tokens_per_s": round(B / (graph_ms * 1e-3), 1),
+                      "gbs": round(step_bytes / (graph_ms * 1e-3) / 1e9, 1), "clocks": graph_clk}}
 
 
 def vicuna13b(stream, peaks, read_gbs, cpu_seconds, with_cpu):

@@ -6,7 +6,9 @@
 // HBM-bound: every cached key and value of the window is read once.
 //
 // Grid: one CTA per (sequence b, head h, split s) where split s covers window
-// entries [s*kChunk, (s+1)*kChunk).  The CTA's 128 threads form row groups of
+// entries [s*CH, (s+1)*CH).  The split size is chosen per launch (see
+// head_chunk): kChunk when the launch has enough splits to fill the GPU,
+// half of it at small batch.  The CTA's 128 threads form row groups of
 // LPR lanes (one 16-byte vector of a cached row per lane); each group walks
 // its share of the chunk in batches of kUnroll rows, issuing the K and V loads
 // of a whole batch together (2*kUnroll 16-byte loads in flight per thread),
@@ -42,8 +44,17 @@ constexpr int kChunk = MOA_DECODE_CHUNK;   // window entries per split (per-head
 constexpr int kGroupChunk = MOA_GQA_CHUNK;
 // Number of splits of x entries, chunk at a time (64-bit, so spans up to
 // INT32_MAX do not wrap).
-__host__ __device__ inline int splits_of(int x, int chunk) { return (int)(((long long)x + chunk - 1) / chunk); }
+__host__ __device__ __forceinline__ int splits_of(int x, int chunk) { return (int)(((long long)x + chunk - 1) / chunk); }
 static_assert(kGroupChunk >= kChunk, "group split size (the workspace holds the per-head kernel's slots)");
+// Per-head split size at small batch.  A launch with fewer than about one
+// wave of CTAs (7 per SM) leaves SMs idle while each CTA streams its long
+// split, so such a launch takes splits of kMinChunk = kChunk / 2 entries
+// instead.  On one Vicuna-7B-shaped layer (32 heads, context 4096, 50 %) a
+// layer took 15.7-15.9 us at batch 1 against 19.0-19.7, 18.3 at batch 2
+// against 22.6 and 24.6 at batch 4 against 26.7; 128- and 64-entry splits
+// were no better.  Larger launches keep kChunk, which measured best there.
+constexpr int kMinChunk = kChunk / 2;
+constexpr long long kHeadItems = 1024;
 constexpr int kUnroll = 4;           // rows per batch: 2*kUnroll 16-byte loads in flight
 // Batches whose rows are contiguous in the ring load from one base pointer at
 // constant offsets (1).  Besides the address arithmetic this frees registers
@@ -130,7 +141,7 @@ __device__ __forceinline__ void step_counted(const DecodeParams& p, int b, int64
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, int CH>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int VE = Vec16<T>::N;     // elements per 16-byte vector
   constexpr int LPR = D / VE;         // lanes per cached row
@@ -165,13 +176,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   if (fused) step_counted(p, b, t0);
   const int64_t tb = fused ? t0 + 1 : t0;              // tokens attended
   const int Seff = (int)(tb < (int64_t)p.span[h] ? tb : (int64_t)p.span[h]);
-  const int nwin = splits_of(p.span[h], kChunk);       // window splits of head h
+  const int nwin = splits_of(p.span[h], CH);           // window splits of head h
   // Splits s >= nwin read the global tokens below the window: positions
   // 0 .. min(k_h, tb - Seff) - 1, at rows of the same index.
   const bool gsplit = s >= nwin;
-  const int w0 = (gsplit ? s - nwin : s) * kChunk;
+  const int w0 = (gsplit ? s - nwin : s) * CH;
   const int nent = gsplit ? (int)min((int64_t)p.sink[h], tb - Seff) : Seff;
-  const int nrows = max(0, min(kChunk, nent - w0));
+  const int nrows = max(0, min(CH, nent - w0));
   const int64_t pos0 = tb - Seff + w0;                 // first window position of this split
   const int slot0 = gsplit ? w0 : nrows > 0 ? (int)(pos0 % C) : 0;
 
@@ -1030,12 +1041,16 @@ cudaError_t launch_group_g(const DecodeParams& p, int G, unsigned grid, cudaStre
 }
 
 template <typename T, int D>
-cudaError_t launch_one(const DecodeParams& p, unsigned grid, cudaStream_t s) {
-  decode_kernel<T, D><<<grid, kDecThreads, 0, s>>>(p);
+cudaError_t launch_one(const DecodeParams& p, int chunk, unsigned grid, cudaStream_t s) {
+  if (chunk == kChunk)
+    decode_kernel<T, D, kChunk><<<grid, kDecThreads, 0, s>>>(p);
+  else
+    decode_kernel<T, D, kMinChunk><<<grid, kDecThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 struct DecodeLayout {
+  int chunk;                         // per-head split size
   int items_per_b;
   size_t ctr_off, bctr_off, ml_off, o_off, total;
 };
@@ -1044,19 +1059,32 @@ struct DecodeLayout {
 // the group kernel sum_h ceil(C_g(h) / chunk); both are at most
 // Hq * ceil(max_h S_h / chunk), which sizes the workspace without knowing the
 // number of KV heads.
+// Per-head splits of one sequence at split size c (window, then global tokens).
+long long head_items(int32_t Hq, const int32_t* spans, const int32_t* sinks, int c) {
+  long long items = 0;
+  for (int h = 0; h < Hq; ++h) items += splits_of(spans[h], c) + (sinks ? splits_of(sinks[h], c) : 0);
+  return items;
+}
+
+// The per-head split size of a launch: kChunk, or kMinChunk when the launch
+// would have fewer than kHeadItems splits.  A function of the shapes alone,
+// so the workspace size and the launch agree.
+int head_chunk(int32_t B, int32_t Hq, const int32_t* spans, const int32_t* sinks) {
+  return (long long)B * head_items(Hq, spans, sinks, kChunk) < kHeadItems ? kMinChunk : kChunk;
+}
+
 DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* spans, const int32_t* sinks) {
   DecodeLayout L;
-  int items = 0, max_s = 0, max_k = 0;
+  L.chunk = head_chunk(B, Hq, spans, sinks);
+  int max_s = 0, max_k = 0;
   for (int h = 0; h < Hq; ++h) {
-    items += splits_of(spans[h], kChunk);
     max_s = max_s > spans[h] ? max_s : spans[h];
-    if (sinks) {
-      items += splits_of(sinks[h], kChunk);   // global-token splits
-      max_k = max_k > sinks[h] ? max_k : sinks[h];
-    }
+    if (sinks) max_k = max_k > sinks[h] ? max_k : sinks[h];
   }
-  L.items_per_b = items;
-  const size_t slots = (size_t)Hq * ((size_t)splits_of(max_s, kChunk) + (size_t)splits_of(max_k, kChunk));
+  L.items_per_b = (int)head_items(Hq, spans, sinks, L.chunk);
+  // The group kernels split more coarsely (kGroupChunk >= chunk), so these
+  // slots hold their partials too.
+  const size_t slots = (size_t)Hq * ((size_t)splits_of(max_s, L.chunk) + (size_t)splits_of(max_k, L.chunk));
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   L.ctr_off = 256;
   L.bctr_off = L.ctr_off + up((size_t)B * Hq * 4);
@@ -1099,7 +1127,7 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   for (int h = 0; h < Hq; ++h) {
     p.span[h] = spans[h];
     p.sink[h] = sinks ? sinks[h] : 0;
-    p.split_pre[h + 1] = p.split_pre[h] + splits_of(spans[h], kChunk) + splits_of(p.sink[h], kChunk);
+    p.split_pre[h + 1] = p.split_pre[h] + splits_of(spans[h], L.chunk) + splits_of(p.sink[h], L.chunk);
   }
   for (int g = 0; g < c->Hkv; ++g) {
     p.cap[g] = c->cap[g];
@@ -1132,7 +1160,11 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
                          (G == 4 || G == 8 || (kGroupMma2 && G == 2));
   if (mma_group || (plain && (G == 4 || G == 8) && head_rows * 10 > group_rows * 22)) {
     // group kernel: splits per KV group over its capacity (then over its
-    // heads' largest global-token count), G partial slots each
+    // heads' largest global-token count), G partial slots each.  Its split
+    // size stays kGroupChunk at every batch: smaller group splits measured
+    // slower even at batch 1 (0.038 against 0.021 ms on a Llama3-8B-shaped
+    // layer), as each warp then gets only a tile or two and the last split
+    // merges many more partials.
     int items = 0;
     p.split_pre[0] = 0;
     p.hslot_pre[0] = 0;
@@ -1163,10 +1195,11 @@ moa_status launch_decode(moa_kv_cache* c, const void* q, void* o, int32_t Hq, co
   if (grid > 0x7fffffffLL) return MOA_ERR_UNSUPPORTED;
   cudaError_t e;
   if (c->dtype == MOA_BF16)
-    e = c->d == 128 ? launch_one<__nv_bfloat16, 128>(p, (unsigned)grid, s)
-                    : launch_one<__nv_bfloat16, 64>(p, (unsigned)grid, s);
+    e = c->d == 128 ? launch_one<__nv_bfloat16, 128>(p, L.chunk, (unsigned)grid, s)
+                    : launch_one<__nv_bfloat16, 64>(p, L.chunk, (unsigned)grid, s);
   else
-    e = c->d == 128 ? launch_one<float, 128>(p, (unsigned)grid, s) : launch_one<float, 64>(p, (unsigned)grid, s);
+    e = c->d == 128 ? launch_one<float, 128>(p, L.chunk, (unsigned)grid, s)
+                    : launch_one<float, 64>(p, L.chunk, (unsigned)grid, s);
   return e == cudaSuccess ? MOA_OK : cuda_fail(e, "decode launch");
 }
 
