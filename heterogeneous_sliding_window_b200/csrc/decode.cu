@@ -1055,10 +1055,6 @@ struct DecodeLayout {
   size_t ctr_off, bctr_off, ml_off, o_off, total;
 };
 
-// Partial slots per sequence: the per-head kernel uses sum_h ceil(S_h / chunk),
-// the group kernel sum_h ceil(C_g(h) / chunk); both are at most
-// Hq * ceil(max_h S_h / chunk), which sizes the workspace without knowing the
-// number of KV heads.
 // Per-head splits of one sequence at split size c (window, then global tokens).
 long long head_items(int32_t Hq, const int32_t* spans, const int32_t* sinks, int c) {
   long long items = 0;
@@ -1073,6 +1069,10 @@ int head_chunk(int32_t B, int32_t Hq, const int32_t* spans, const int32_t* sinks
   return (long long)B * head_items(Hq, spans, sinks, kChunk) < kHeadItems ? kMinChunk : kChunk;
 }
 
+// Partial slots per sequence: the per-head kernel uses sum_h ceil(S_h / chunk),
+// the group kernel sum_h ceil(C_g(h) / chunk); both are at most
+// Hq * ceil(max_h S_h / chunk), which sizes the workspace without knowing the
+// number of KV heads.
 DecodeLayout decode_layout(int32_t B, int32_t Hq, int32_t d, const int32_t* spans, const int32_t* sinks) {
   DecodeLayout L;
   L.chunk = head_chunk(B, Hq, spans, sinks);
