@@ -561,6 +561,43 @@ def test_bf16_decode_vicuna7b_layer_full_size_sampled():
         assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
 
 
+@pytest.mark.parametrize("B", [1, 4])
+def test_bf16_decode_vicuna7b_layer_small_batch(B):
+    """The same layer at batch 1 and 4, where the launch has under 1 024 splits of 512 entries
+    and the kernel takes half-size splits (up to 16 per head here): every head, fused append,
+    against the oracle's ring decode; the appended rows bit-exact."""
+    H, d, N = 32, 128, 4096
+    a, b = inputs.tables_7b(1000, H, N, 64, 0.5, orules.eval_spans)
+    spans = moa.moa_rules_eval(a, b, N, 64)
+    cache = moa.KVCache(B, H, d, "bf16", spans)
+    data = cache.data_bytes().view(torch.bfloat16)
+    data.copy_(inputs.randn_cuda(15 + B, (data.numel(),)))
+    cache.set_positions([N] * B)
+    host = cache.data_bytes().cpu().numpy().tobytes()
+    scale = 1.0 / math.sqrt(d)
+    qt = inputs.randn_cuda(16 + B, (B, H, d))
+    kt = inputs.randn_cuda(17 + B, (B, H, 1, d))
+    vt = inputs.randn_cuda(18 + B, (B, H, 1, d))
+    ws = moa.Workspace(moa.MOA_OP_DECODE, B, H, 0, d, spans)
+    ot = _nan_like((B, H, d), torch.bfloat16)
+    moa.moa_decode_append(cache.handle, qt, kt, vt, ot, H, spans, scale, ws.ptr, ws.nbytes)
+    moa.moa_workspace_check(ws.ptr)
+    torch.cuda.synchronize()
+    assert cache.positions() == [N + 1] * B
+    after = cache.data_bytes().cpu().numpy().tobytes()
+    kt64, vt64, qt64, ot64 = (inputs.as_f64(x) for x in (kt, vt, qt, ot))
+    for bb in range(B):
+        for hh in range(H):
+            K, V = okv.block_from_image(host, bb, hh, B, H, d, spans, "bf16")
+            C = spans[hh]
+            K[N % C] = kt64[bb, hh, 0]      # the appended token's slot
+            V[N % C] = vt64[bb, hh, 0]
+            K2, V2 = okv.block_from_image(after, bb, hh, B, H, d, spans, "bf16")
+            assert np.array_equal(K2[N % C], K[N % C]) and np.array_equal(V2[N % C], V[N % C]), (bb, hh)
+            ref = okv.decode_row_from_ring(K, V, N + 1, spans[hh], qt64[bb, hh], scale)
+            assert np.max(np.abs(ot64[bb, hh] - ref)) <= BF16_TOL, (bb, hh)
+
+
 def test_bf16_decode_llama3_gqa_layer_full_size_sampled():
     """A Llama3-8B-shaped GQA decode layer: B=4, 32 query heads on 8 KV heads, context 8192,
     per-head spans at 50% density (heterogeneous within each group), one appended token."""
