@@ -340,17 +340,57 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   if (!last_flag) return;
   __threadfence();
   const size_t first = (size_t)b * p.items_per_b + p.split_pre[h];
-  float MM = -INFINITY;
-  for (int ss = 0; ss < nsplit; ++ss) MM = fmaxf(MM, __ldcg(&p.part_ml[2 * (first + ss)]));
-  float LL = 0.f, A = 0.f;
+  // Merge of the splits' partials by the whole CTA: the maximum and the
+  // denominator are reduced over the threads, and each output column sums
+  // its splits in four independent chains, so the loads overlap.  A serial
+  // walk over the splits would put one L2 round trip per split on the tail
+  // of the launch, which at small batch is its critical path.
+  __shared__ float w_sh[kDecThreads];
+  __shared__ float red[kDecWarps];
+  float mx = -INFINITY;
+  for (int ss = tid; ss < nsplit; ss += kDecThreads) mx = fmaxf(mx, __ldcg(&p.part_ml[2 * (first + ss)]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  float MM = red[0];
+#pragma unroll
+  for (int k = 1; k < kDecWarps; ++k) MM = fmaxf(MM, red[k]);
+  __syncthreads();                                 // red is reused for the denominator
+  float ll = 0.f, A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f;
   if (MM != -INFINITY) {
-    for (int ss = 0; ss < nsplit; ++ss) {
-      const float ms = __ldcg(&p.part_ml[2 * (first + ss)]);
-      const float w = exp2f(ms - MM);              // 0 for empty splits (ms = -inf)
-      LL = fmaf(w, __ldcg(&p.part_ml[2 * (first + ss) + 1]), LL);
-      if (tid < D) A = fmaf(w, __ldcg(&p.part_o[(first + ss) * D + tid]), A);
+    for (int base = 0; base < nsplit; base += kDecThreads) {
+      const int ss = base + tid;
+      float w = 0.f;
+      if (ss < nsplit) {
+        w = exp2f(__ldcg(&p.part_ml[2 * (first + ss)]) - MM);   // 0 for empty splits (m = -inf)
+        ll = fmaf(w, __ldcg(&p.part_ml[2 * (first + ss) + 1]), ll);
+      }
+      w_sh[tid] = w;
+      __syncthreads();
+      const int n = min(kDecThreads, nsplit - base);
+      if (tid < D) {
+        const float* po = p.part_o + (first + base) * D + tid;
+        int k = 0;
+        for (; k + 3 < n; k += 4) {
+          A0 = fmaf(w_sh[k], __ldcg(po + (size_t)k * D), A0);
+          A1 = fmaf(w_sh[k + 1], __ldcg(po + (size_t)(k + 1) * D), A1);
+          A2 = fmaf(w_sh[k + 2], __ldcg(po + (size_t)(k + 2) * D), A2);
+          A3 = fmaf(w_sh[k + 3], __ldcg(po + (size_t)(k + 3) * D), A3);
+        }
+        for (; k < n; ++k) A0 = fmaf(w_sh[k], __ldcg(po + (size_t)k * D), A0);
+      }
+      __syncthreads();
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+  if ((tid & 31) == 0) red[tid >> 5] = ll;
+  __syncthreads();
+  float LL = 0.f;
+#pragma unroll
+  for (int k = 0; k < kDecWarps; ++k) LL += red[k];
+  const float A = (A0 + A1) + (A2 + A3);
   if (tid < D) Vec16<T>::store(out + tid, LL > 0.f ? A / LL : 0.f);
   if (tid == 0) {
     p.ctr[(size_t)b * p.Hq + h] = 0u;
