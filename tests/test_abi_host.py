@@ -276,6 +276,20 @@ def test_workspace_sizes():
         moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 2, 4, 0, 128, [64, 0, 1, 1])
 
 
+def test_decode_workspace_holds_the_small_batch_splits():
+    """A decode launch with under 1 024 splits of 512 entries takes 256-entry splits, so its
+    workspace must hold twice as many partials (m, l and d floats each) as 512-entry splits."""
+    d, Hq = 128, 32
+    spans = [4096] * Hq                           # 8 splits of 512 per head
+    def partial_bytes(B, chunk):
+        return B * Hq * (-(-4096 // chunk)) * (d + 2) * 4
+    small = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 1, Hq, 0, d, spans)       # 256 at 512: half-size splits
+    large = moa.moa_workspace_bytes(moa.MOA_OP_DECODE, 32, Hq, 0, d, spans)      # 8192 at 512
+    assert small >= partial_bytes(1, 256)
+    assert large >= partial_bytes(32, 512)
+    assert large < partial_bytes(32, 256)          # large launches keep 512-entry splits
+
+
 def test_input_tables_reach_target_density():
     """The seeded table generator lands near the requested mean span / N."""
     for density, N in [(0.25, 8192), (0.5, 4096), (0.125, 32768)]:
